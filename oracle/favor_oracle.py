@@ -1,0 +1,262 @@
+"""FAVOR attention oracle: a plain, slow fp64 CPU implementation.
+
+TEST INFRASTRUCTURE ONLY. Only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline
+and reference legs may import this module. The CUDA library never calls it and shares no
+code with it. Inputs reach both sides from the ``favor_inputs`` generator alone.
+
+Sources (page title, section):
+  [EXPL] "用随机特征“骗”过 softmax，Transformer 注意力也能跑成线性？" (explainer of arXiv 2009.14794),
+         section "核心机制：FAVOR+". Covers:
+         - Att = D^-1 A V with A = exp(QK^T/sqrt(d));
+         - exp(q^T k/sqrt(d)) ~ phi(q)^T phi(k);
+         - phi(K)^T V aggregated first (an m x v state), then left-multiplied by phi(Q);
+         - D_hat = phi(Q)(phi(K)^T 1);
+         - the trigonometric mode (cos/sin pairs, from Rahimi-Recht random Fourier features);
+         - ORF directions;
+         - the causal prefix sum of phi(k_j) v_j^T over j <= i.
+  [MLMP-zh] "Masked Language Modeling for Proteins via Linearly Scalable Long-Context
+         Transformers" (gptget.net, Chinese), sections "方法详解" and "核心创新"
+         (Gaussian-kernel random features, ORF, prefix sum, generalized attention),
+         and "实验设计" (orthogonal vs unstructured ablation).
+  [MLMP-en] the same title (gptget.net, English), sections "Methodology" and
+         "AI Executive Summary" (Gaussian kernel random features, orthogonal sampling).
+
+Readings where the pages are silent:
+  * Trig map. phi(x) = exp(|x|^2/2)/sqrt(M) * [cos(w_1.x) .. cos(w_M.x), sin(w_1.x) .. sin(w_M.x)].
+    This is the random Fourier feature map of the Gaussian kernel, times exp(|x|^2/2),
+    because exp(q.k) = exp(|q|^2/2) exp(-|q-k|^2/2) exp(|k|^2/2).
+  * ReLU (generalized attention) map. phi(x) = max(Omega x, 0)/sqrt(M).
+  * Temperature. The 1/sqrt(d) is carried by the inputs (Q and K pre-scaled by
+    d^-1/4). Nothing here rescales.
+  * ORF. ceil(M/d) blocks of d x d Gaussians, rows orthonormalised in order
+    (Gram-Schmidt, equivalently QR with a positive R diagonal). Row r is then scaled by
+    the length of an independent N(0, I_d) vector (chi_d), the blocks are stacked,
+    and the result is cut to M rows.
+  * A zero denominator gives a zero output row. A negative trig denominator is used
+    as is.
+Every factor is kept in fp64. There is no stabiliser, and exp(|x|^2/2) is finite
+for |x|^2/2 < 709.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+TRIG = 0
+RELU = 1
+
+
+# ---------------------------------------------------------------- random matrices
+def gram_schmidt_rows(G: np.ndarray) -> np.ndarray:
+    """Orthonormalise the rows of a square block in order.
+
+    Classical Gram-Schmidt, applied twice per row ("twice is enough"), so the rows are
+    orthonormal to fp64 rounding. [EXPL, 核心机制] constrains the directions to a random
+    subsample of an orthogonal matrix, and [MLMP-zh, 方法详解] calls them orthogonal
+    random features.
+    """
+    Q = np.array(G, dtype=np.float64, copy=True)
+    for i in range(Q.shape[0]):
+        v = Q[i].copy()
+        for _ in range(2):
+            if i:
+                v = v - Q[:i].T @ (Q[:i] @ v)
+        Q[i] = v / np.linalg.norm(v)
+    return Q
+
+
+def orf_matrix(G: np.ndarray, R: np.ndarray, M: int) -> np.ndarray:
+    """ORF Omega [M, d] for one head.
+
+    G [nb, d, d] holds the Gaussian blocks and R [M, d] the chi draws. Each block is
+    orthonormalised, row r is scaled by |R[r]|, the blocks are stacked and the result
+    is cut to M rows.
+    """
+    blocks = [gram_schmidt_rows(G[i]) for i in range(G.shape[0])]
+    Q = np.concatenate(blocks, axis=0)[:M]
+    return Q * np.linalg.norm(R, axis=1)[:, None]
+
+
+def orf_matrices(G: np.ndarray, R: np.ndarray, M: int) -> np.ndarray:
+    """Per-head ORF matrices: G [H, nb, d, d], R [H, M, d] -> Omega [H, M, d]."""
+    return np.stack([orf_matrix(G[h], R[h], M) for h in range(G.shape[0])])
+
+
+# ---------------------------------------------------------------- feature maps
+def phi_trig(X: np.ndarray, Om: np.ndarray) -> np.ndarray:
+    """Trigonometric softmax-kernel features [L, 2M] of the rows of X [L, d].
+
+    [EXPL, 核心机制]: cos/sin pairs from random Fourier features. [MLMP-en, AI Executive
+    Summary]: random features of the Gaussian kernel. The exp(|x|^2/2) factor turns the
+    Gaussian kernel into exp(q.k).
+    """
+    M = Om.shape[0]
+    U = X @ Om.T
+    g = np.exp(0.5 * np.sum(X * X, axis=1)) / np.sqrt(M)
+    return g[:, None] * np.concatenate([np.cos(U), np.sin(U)], axis=1)
+
+
+def phi_relu(X: np.ndarray, Om: np.ndarray) -> np.ndarray:
+    """Generalized-attention ReLU features [L, M]: max(Omega x, 0)/sqrt(M).
+
+    [MLMP-zh, 核心创新] names generalized kernel attention (GA). The ReLU map is the GA
+    kernel this library implements.
+    """
+    return np.maximum(X @ Om.T, 0.0) / np.sqrt(Om.shape[0])
+
+
+def phi(X: np.ndarray, Om: np.ndarray, kind: int) -> np.ndarray:
+    if kind == TRIG:
+        return phi_trig(X, Om)
+    if kind == RELU:
+        return phi_relu(X, Om)
+    raise ValueError(f"unknown feature kind {kind}")
+
+
+def _normalise(num: np.ndarray, den: np.ndarray) -> np.ndarray:
+    out = np.zeros_like(num)
+    nz = den != 0.0
+    out[nz] = num[nz] / den[nz, None]
+    return out
+
+
+# ---------------------------------------------------------------- one head
+def favor_bidirectional_head(q, k, v, Om, kind):
+    """Bidirectional FAVOR for one head, in linear time.
+
+    [EXPL, 核心机制]: aggregate S = phi(K)^T V and z = phi(K)^T 1 first, then
+    out = D_hat^-1 phi(Q) S with D_hat = diag(phi(Q) z). No L x L matrix is formed.
+    """
+    fq = phi(q, Om, kind)
+    fk = phi(k, Om, kind)
+    S = fk.T @ v
+    z = fk.T @ np.ones(k.shape[0])
+    return _normalise(fq @ S, fq @ z)
+
+
+def favor_causal_head(q, k, v, Om, kind):
+    """Causal FAVOR for one head, as a sequential fp64 prefix loop.
+
+    [EXPL, 核心机制]: the state sum_{j<=i} phi(k_j) v_j^T and its normaliser
+    sum_{j<=i} phi(k_j) are accumulated in order. Row i reads the state after
+    token i is added.
+    """
+    fq = phi(q, Om, kind)
+    fk = phi(k, Om, kind)
+    L, dv = v.shape
+    S = np.zeros((fk.shape[1], dv))
+    z = np.zeros(fk.shape[1])
+    out = np.zeros((L, dv))
+    for i in range(L):
+        S += np.outer(fk[i], v[i])
+        z += fk[i]
+        den = fq[i] @ z
+        if den != 0.0:
+            out[i] = (fq[i] @ S) / den
+    return out
+
+
+def favor_explicit_head(q, k, v, Om, kind, causal, rows=None):
+    """The quadratic form D_hat^-1 A_hat V with A_hat = phi(Q) phi(K)^T, for chosen rows.
+
+    [EXPL, 核心机制]: the estimate of A whose reassociation gives the linear-time form.
+    Causal keeps j <= i only.
+    """
+    rows = np.arange(q.shape[0]) if rows is None else np.asarray(rows)
+    A = phi(q[rows], Om, kind) @ phi(k, Om, kind).T
+    if causal:
+        A = np.where(np.arange(k.shape[0])[None, :] <= rows[:, None], A, 0.0)
+    return _normalise(A @ v, A.sum(axis=1))
+
+
+def softmax_attention_head(q, k, v, causal, rows=None):
+    """Exact softmax attention D^-1 A V with A = exp(q_i . k_j) ([EXPL, 核心机制]).
+
+    The inputs carry the 1/sqrt(d) temperature. Rows are shifted by their max before
+    the exponential.
+    """
+    rows = np.arange(q.shape[0]) if rows is None else np.asarray(rows)
+    s = q[rows] @ k.T
+    if causal:
+        s = np.where(np.arange(k.shape[0])[None, :] <= rows[:, None], s, -np.inf)
+    s = s - s.max(axis=1, keepdims=True)
+    a = np.exp(s)
+    return (a @ v) / a.sum(axis=1, keepdims=True)
+
+
+def arccos_attention_head(q, k, v, causal, rows=None):
+    """The ReLU map's M -> infinity limit: attention with the degree-1 arc-cosine kernel.
+
+    E[relu(w.q) relu(w.k)] over w ~ N(0, I) is |q||k|(sin t + (pi - t) cos t)/(2 pi), with
+    t the angle between q and k (Cho & Saul 2009). ORF rows have the same N(0, I)
+    marginal. Used only to check convergence in M.
+    """
+    rows = np.arange(q.shape[0]) if rows is None else np.asarray(rows)
+    qs = q[rows]
+    nq = np.linalg.norm(qs, axis=1)[:, None]
+    nk = np.linalg.norm(k, axis=1)[None, :]
+    c = np.clip((qs @ k.T) / (nq * nk), -1.0, 1.0)
+    t = np.arccos(c)
+    A = nq * nk * (np.sin(t) + (np.pi - t) * c) / (2 * np.pi)
+    if causal:
+        A = np.where(np.arange(k.shape[0])[None, :] <= rows[:, None], A, 0.0)
+    return _normalise(A @ v, A.sum(axis=1))
+
+
+def row_diagnostics_head(q, k, v, Om, kind, causal, rows=None):
+    """Cancellation diagnostics for chosen rows of the FAVOR estimate.
+
+    kappa_i = sum_j |a_ij| / |sum_j a_ij|  (1 for the ReLU map)
+    s_i     = sum_j |a_ij| * max|v_j| / |sum_j a_ij|
+    a_ij = phi(q_i).phi(k_j). Causal keeps j <= i.
+    """
+    rows = np.arange(q.shape[0]) if rows is None else np.asarray(rows)
+    A = phi(q[rows], Om, kind) @ phi(k, Om, kind).T
+    if causal:
+        A = np.where(np.arange(k.shape[0])[None, :] <= rows[:, None], A, 0.0)
+    absA = np.abs(A)
+    den = np.abs(A.sum(axis=1))
+    with np.errstate(divide="ignore", invalid="ignore"):
+        kappa = absA.sum(axis=1) / den
+        s = (absA @ np.abs(v).max(axis=1)) / den
+    return kappa, s
+
+
+# ---------------------------------------------------------------- [B, H, L, d] wrappers
+def _per_head(fn, Q, K, V, Om, *args, **kw):
+    B, H = Q.shape[:2]
+    out = None
+    for b in range(B):
+        for h in range(H):
+            o = fn(Q[b, h], K[b, h], V[b, h], Om[h], *args, **kw)
+            if out is None:
+                out = np.zeros((B, H) + o.shape)
+            out[b, h] = o
+    return out
+
+
+def favor_attention(Q, K, V, Om, kind, causal):
+    """FAVOR forward for Q, K, V [B, H, L, d] and Omega [H, M, d] (fp64 arrays)."""
+    fn = favor_causal_head if causal else favor_bidirectional_head
+    return _per_head(fn, Q, K, V, Om, kind)
+
+
+def favor_explicit(Q, K, V, Om, kind, causal, rows=None):
+    return _per_head(favor_explicit_head, Q, K, V, Om, kind, causal, rows)
+
+
+def softmax_attention(Q, K, V, causal, rows=None):
+    B, H = Q.shape[:2]
+    return np.stack([np.stack([softmax_attention_head(Q[b, h], K[b, h], V[b, h], causal, rows)
+                               for h in range(H)]) for b in range(B)])
+
+
+def row_diagnostics(Q, K, V, Om, kind, causal, rows=None):
+    B, H = Q.shape[:2]
+    kap, s = [], []
+    for b in range(B):
+        for h in range(H):
+            a, c = row_diagnostics_head(Q[b, h], K[b, h], V[b, h], Om[h], kind, causal, rows)
+            kap.append(a)
+            s.append(c)
+    L_rows = kap[0].shape[0]
+    return np.stack(kap).reshape(B, H, L_rows), np.stack(s).reshape(B, H, L_rows)

@@ -1,0 +1,92 @@
+"""Planted mistakes in the oracle must trip at least one pin.
+
+Each case patches one oracle function (on the CPU, for the duration of the test) with a
+plausible slip, then runs the pins that should catch it and expects an AssertionError.
+"""
+import numpy as np
+import pytest
+
+from oracle import favor_oracle as O
+import test_oracle_pins as P
+
+
+def _phi_trig_no_exp(X, Om):
+    U = X @ Om.T
+    return np.concatenate([np.cos(U), np.sin(U)], axis=1) / np.sqrt(Om.shape[0])
+
+
+def _phi_trig_cos_twice(X, Om):
+    U = X @ Om.T
+    g = np.exp(0.5 * np.sum(X * X, axis=1)) / np.sqrt(Om.shape[0])
+    return g[:, None] * np.concatenate([np.cos(U), np.cos(U)], axis=1)
+
+
+def _phi_trig_sign_slip(X, Om):
+    U = X @ Om.T
+    g = np.exp(0.5 * np.sum(X * X, axis=1)) / np.sqrt(Om.shape[0])
+    return g[:, None] * np.concatenate([np.cos(U), np.sin(-np.abs(U))], axis=1)
+
+
+def _phi_relu_no_max(X, Om):
+    return (X @ Om.T) / np.sqrt(Om.shape[0])
+
+
+def _causal_strict(q, k, v, Om, kind):
+    fq, fk = O.phi(q, Om, kind), O.phi(k, Om, kind)
+    S = np.zeros((fk.shape[1], v.shape[1]))
+    z = np.zeros(fk.shape[1])
+    out = np.zeros_like(v)
+    for i in range(q.shape[0]):
+        den = fq[i] @ z
+        if den != 0:
+            out[i] = (fq[i] @ S) / den
+        S += np.outer(fk[i], v[i])
+        z += fk[i]
+    return out
+
+
+def _bidir_wrong_normaliser(q, k, v, Om, kind):
+    fq, fk = O.phi(q, Om, kind), O.phi(k, Om, kind)
+    return (fq @ (fk.T @ v)) / fq.sum(axis=1, keepdims=True)
+
+
+def _gs_no_normalise(G):
+    Q = np.array(G, dtype=np.float64, copy=True)
+    for i in range(1, Q.shape[0]):
+        Q[i] = Q[i] - Q[:i].T @ ((Q[:i] @ Q[i]) / np.sum(Q[:i] * Q[:i], axis=1))
+    return Q
+
+
+def _orf_no_chi(G, R, M):
+    return np.concatenate([O.gram_schmidt_rows(G[i]) for i in range(G.shape[0])], axis=0)[:M]
+
+
+def _softmax_mask_slip(q, k, v, causal, rows=None):
+    rows = np.arange(q.shape[0]) if rows is None else np.asarray(rows)
+    s = q[rows] @ k.T
+    if causal:
+        s = np.where(np.arange(k.shape[0])[None, :] < rows[:, None] + 2, s, -np.inf)
+    a = np.exp(s - s.max(axis=1, keepdims=True))
+    return (a @ v) / a.sum(axis=1, keepdims=True)
+
+
+CASES = [
+    ("phi_trig", _phi_trig_no_exp, [P.test_trig_self_inner_product_identity]),
+    ("phi_trig", _phi_trig_cos_twice, [P.test_trig_self_inner_product_identity]),
+    ("phi_trig", _phi_trig_sign_slip, [P.test_trig_cross_term_closed_form]),
+    ("phi_relu", _phi_relu_no_max, [lambda: P.test_relu_outputs_are_convex_combinations(False)]),
+    ("favor_causal_head", _causal_strict, [lambda: P.test_causal_prefix_equals_masked(O.TRIG)]),
+    ("favor_bidirectional_head", _bidir_wrong_normaliser,
+     [lambda: P.test_linear_equals_explicit_bidirectional(O.TRIG)]),
+    ("gram_schmidt_rows", _gs_no_normalise, [P.test_gram_schmidt_matches_qr_with_positive_diagonal]),
+    ("orf_matrix", _orf_no_chi, [lambda: P.test_orf_structure(32, 16)]),
+    ("softmax_attention_head", _softmax_mask_slip, [lambda: P.test_softmax_matches_torch(True)]),
+]
+
+
+@pytest.mark.parametrize("name,bad,pins", CASES, ids=[f"{c[0]}:{c[1].__name__}" for c in CASES])
+def test_planted_mistake_is_caught(monkeypatch, name, bad, pins):
+    monkeypatch.setattr(O, name, bad)
+    for pin in pins:
+        with pytest.raises((AssertionError, ValueError, FloatingPointError)):
+            pin()

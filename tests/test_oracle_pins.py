@@ -1,0 +1,281 @@
+"""Pins for the fp64 oracle, each against something other than the oracle itself.
+
+What pins what:
+  * exact softmax attention          -> torch.softmax (library special case), brute force
+  * trig features                    -> the identity cos^2 + sin^2 = 1, the cosine-difference
+                                        identity, a scalar closed form
+  * bidirectional linear form        -> the explicit quadratic form D_hat^-1 A_hat V
+  * causal prefix loop               -> the masked quadratic form, row 0 = v_0,
+                                        last row = bidirectional last row
+  * invariants                       -> constant V, linearity in V, joint (k, v)
+                                        permutation, permutation of Omega rows, ReLU convexity
+  * ORF                              -> QR with a positive R diagonal (numpy.linalg.qr),
+                                        orthogonality, chi norms, N(0, I) marginal
+  * unbiasedness / variance / M      -> Gaussian characteristic function,
+                                        arc-cosine kernel, closed-form i.i.d. variance
+The pages print no worked example, so no stored page value pins the oracle.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import favor_inputs as fi
+from oracle import favor_oracle as O
+
+
+def _qkv(L, d, seed=0, B=1, H=1):
+    q, k, v = fi.qkv(B, H, L, d, seed=seed)
+    return q.astype(np.float64)[0, 0], k.astype(np.float64)[0, 0], v.astype(np.float64)[0, 0]
+
+
+def _orf(M, d, seed=0, H=1):
+    G, R = fi.orf_gaussians(H, M, d, seed=seed)
+    return O.orf_matrices(G, R, M)
+
+
+# ------------------------------------------------------------------ exact softmax
+@pytest.mark.parametrize("causal", [False, True])
+def test_softmax_matches_torch(causal):
+    q, k, v = _qkv(37, 8, seed=3)
+    got = O.softmax_attention_head(q, k, v, causal)
+    s = torch.from_numpy(q) @ torch.from_numpy(k).T
+    if causal:
+        s = s.masked_fill(torch.triu(torch.ones(37, 37, dtype=torch.bool), 1), float("-inf"))
+    ref = torch.softmax(s, dim=-1) @ torch.from_numpy(v)
+    np.testing.assert_allclose(got, ref.numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_softmax_bruteforce_tiny():
+    q = np.array([[0.3, -1.0], [2.0, 0.5], [-0.7, 0.1]])
+    k = np.array([[1.0, 0.0], [0.2, -0.4], [0.0, 1.5]])
+    v = np.array([[1.0, 2.0, 3.0], [-1.0, 0.0, 4.0], [0.5, 0.5, -2.0]])
+    for causal in (False, True):
+        exp_out = np.zeros((3, 3))
+        for i in range(3):
+            w = [math.exp(sum(q[i, t] * k[j, t] for t in range(2))) if (not causal or j <= i) else 0.0
+                 for j in range(3)]
+            for c in range(3):
+                exp_out[i, c] = sum(w[j] * v[j, c] for j in range(3)) / sum(w)
+        np.testing.assert_allclose(O.softmax_attention_head(q, k, v, causal), exp_out, rtol=1e-13)
+    # rows of D^-1 A sum to one: V = ones gives ones
+    np.testing.assert_allclose(O.softmax_attention_head(q, k, np.ones((3, 2)), False), 1.0, rtol=1e-14)
+
+
+# ------------------------------------------------------------------ feature maps
+def test_trig_self_inner_product_identity():
+    x, _, _ = _qkv(50, 16, seed=1)
+    x = x * 2.5
+    om = np.random.default_rng(5).standard_normal((24, 16)) * 3.0  # any Omega works
+    f = O.phi_trig(x, om)
+    np.testing.assert_allclose(np.sum(f * f, axis=1), np.exp(np.sum(x * x, axis=1)), rtol=1e-12)
+
+
+def test_trig_cross_term_closed_form():
+    q, k, _ = _qkv(20, 16, seed=2)
+    om = _orf(32, 16, seed=4)[0]
+    got = O.phi_trig(q, om) @ O.phi_trig(k, om).T
+    nq = np.sum(q * q, axis=1)[:, None]
+    nk = np.sum(k * k, axis=1)[None, :]
+    diff = q[:, None, :] - k[None, :, :]                       # [20, 20, d]
+    mean_cos = np.cos(np.einsum("ijd,md->ijm", diff, om)).mean(axis=2)
+    np.testing.assert_allclose(got, np.exp(0.5 * (nq + nk)) * mean_cos, rtol=1e-11, atol=1e-300)
+
+
+def test_scalar_closed_form_trig():
+    # d = 1, M = 1: a_ij = exp((q_i^2 + k_j^2)/2) cos(w (q_i - k_j)), worked by hand
+    w = 0.8
+    q = np.array([[0.4], [-1.1], [0.25]])
+    k = np.array([[0.9], [-0.3], [0.0]])
+    v = np.array([[1.0, -2.0], [0.5, 3.0], [-1.5, 0.25]])
+    a = np.array([[math.exp((qi * qi + kj * kj) / 2) * math.cos(w * (qi - kj)) for kj in k[:, 0]]
+                  for qi in q[:, 0]])
+    bid = (a @ v) / a.sum(axis=1, keepdims=True)
+    al = np.tril(a)
+    cau = (al @ v) / al.sum(axis=1, keepdims=True)
+    om = np.array([[w]])
+    np.testing.assert_allclose(O.favor_bidirectional_head(q, k, v, om, O.TRIG), bid, rtol=1e-12)
+    np.testing.assert_allclose(O.favor_causal_head(q, k, v, om, O.TRIG), cau, rtol=1e-12)
+
+
+def test_small_closed_form_relu():
+    # Omega = I_2 plus the row (1, -1): phi(x) = (max(x1,0), max(x2,0), max(x1-x2,0))/sqrt(3)
+    om = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, -1.0]])
+    q = np.array([[1.0, 2.0], [-1.0, 0.5]])
+    k = np.array([[2.0, 1.0], [0.5, -1.0], [-3.0, 4.0]])
+    v = np.array([[1.0], [2.0], [4.0]])
+    f = lambda x: np.array([max(x[0], 0), max(x[1], 0), max(x[0] - x[1], 0)]) / math.sqrt(3)
+    a = np.array([[f(qi) @ f(kj) for kj in k] for qi in q])
+    # q0 = (1,2): f = (1,2,0)/sqrt3. k0: (2,1,1)/sqrt3 -> 4/3, k1: (.5,0,1.5)/sqrt3 -> .5/3, k2: (0,4,0)/sqrt3 -> 8/3
+    np.testing.assert_allclose(a[0], [4 / 3, 0.5 / 3, 8 / 3], rtol=1e-14)
+    bid = (a @ v)[:, 0] / a.sum(axis=1)
+    np.testing.assert_allclose(O.favor_bidirectional_head(q, k, v, om, O.RELU)[:, 0], bid, rtol=1e-13)
+
+
+# ------------------------------------------------------------------ reassociation and causal prefix
+@pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
+def test_linear_equals_explicit_bidirectional(kind):
+    q, k, v = _qkv(256, 16, seed=0)
+    om = _orf(32, 16, seed=0)[0]
+    lin = O.favor_bidirectional_head(q, k, v, om, kind)
+    exp_ = O.favor_explicit_head(q, k, v, om, kind, causal=False)
+    np.testing.assert_allclose(lin, exp_, rtol=1e-9, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
+def test_causal_prefix_equals_masked(kind):
+    q, k, v = _qkv(200, 16, seed=1)
+    om = _orf(32, 16, seed=1)[0]
+    cau = O.favor_causal_head(q, k, v, om, kind)
+    np.testing.assert_allclose(cau, O.favor_explicit_head(q, k, v, om, kind, causal=True),
+                               rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(cau[0], v[0], rtol=1e-12)
+    np.testing.assert_allclose(cau[-1], O.favor_bidirectional_head(q, k, v, om, kind)[-1], rtol=1e-10)
+
+
+# ------------------------------------------------------------------ invariants
+@pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
+@pytest.mark.parametrize("causal", [False, True])
+def test_invariants(kind, causal):
+    q, k, v = _qkv(96, 16, seed=7)
+    om = _orf(32, 16, seed=7)[0]
+    f = O.favor_causal_head if causal else O.favor_bidirectional_head
+    c = np.linspace(-1.0, 2.0, 16)
+    np.testing.assert_allclose(f(q, k, np.tile(c, (96, 1)), om, kind), np.tile(c, (96, 1)), rtol=1e-9)
+    v2 = np.random.default_rng(1).standard_normal(v.shape)
+    np.testing.assert_allclose(f(q, k, 2.0 * v - 3.0 * v2, om, kind),
+                               2.0 * f(q, k, v, om, kind) - 3.0 * f(q, k, v2, om, kind), rtol=1e-9, atol=1e-11)
+    perm = np.random.default_rng(2).permutation(32)
+    np.testing.assert_allclose(f(q, k, v, om[perm], kind), f(q, k, v, om, kind), rtol=1e-9, atol=1e-12)
+    if not causal:
+        p = np.random.default_rng(3).permutation(96)
+        np.testing.assert_allclose(f(q, k[p], v[p], om, kind), f(q, k, v, om, kind), rtol=1e-9, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_relu_outputs_are_convex_combinations(causal):
+    q, k, v = _qkv(128, 16, seed=9)
+    om = _orf(32, 16, seed=9)[0]
+    out = (O.favor_causal_head if causal else O.favor_bidirectional_head)(q, k, v, om, O.RELU)
+    for i in range(128):
+        vv = v[: i + 1] if causal else v
+        assert np.all(out[i] >= vv.min(axis=0) - 1e-12) and np.all(out[i] <= vv.max(axis=0) + 1e-12)
+    kap, _ = O.row_diagnostics_head(q, k, v, om, O.RELU, causal)
+    np.testing.assert_allclose(kap, 1.0, rtol=1e-12)
+
+
+def test_zero_denominator_gives_zero_row():
+    om = np.array([[1.0, 0.0], [0.0, 1.0]])
+    q = np.array([[-1.0, -1.0], [1.0, 1.0]])        # phi_relu(q0) = 0
+    k = np.array([[1.0, 2.0], [3.0, 0.5]])
+    v = np.array([[1.0, 1.0], [2.0, -1.0]])
+    out = O.favor_bidirectional_head(q, k, v, om, O.RELU)
+    assert np.all(out[0] == 0.0) and np.all(np.isfinite(out))
+
+
+# ------------------------------------------------------------------ ORF
+def test_gram_schmidt_matches_qr_with_positive_diagonal():
+    G = np.random.default_rng(11).standard_normal((64, 64))
+    Qr, Rr = np.linalg.qr(G.T)          # G^T = Qr Rr, columns of Qr = rows orthonormalised in order
+    Qr = Qr * np.sign(np.diag(Rr))[None, :]
+    np.testing.assert_allclose(O.gram_schmidt_rows(G), Qr.T, atol=1e-11)
+
+
+@pytest.mark.parametrize("M,d", [(32, 16), (256, 64), (40, 16)])
+def test_orf_structure(M, d):
+    G, R = fi.orf_gaussians(1, M, d, seed=5)
+    om = O.orf_matrix(G[0], R[0], M)
+    assert om.shape == (M, d)
+    norms = np.linalg.norm(om, axis=1)
+    np.testing.assert_allclose(norms, np.linalg.norm(R[0], axis=1), rtol=1e-12)
+    unit = om / norms[:, None]
+    for b0 in range(0, M, d):
+        blk = unit[b0:b0 + d]
+        np.testing.assert_allclose(blk @ blk.T, np.eye(blk.shape[0]), atol=1e-12)
+    # the rows come from the blocks in order, the last block cut when d does not divide M
+    np.testing.assert_allclose(unit[:d], O.gram_schmidt_rows(G[0, 0]), atol=1e-13)
+
+
+def test_orf_row_marginal_is_standard_normal():
+    d, M, n = 8, 16, 3000
+    rows = []
+    for s in range(n):
+        G, R = fi.orf_gaussians(1, M, d, seed=1000 + s)
+        rows.append(O.orf_matrix(G[0], R[0], M))
+    W = np.concatenate(rows)                      # n*M rows
+    cov = W.T @ W / W.shape[0]
+    np.testing.assert_allclose(cov, np.eye(d), atol=0.05)
+    chi_mean = math.sqrt(2) * math.exp(math.lgamma((d + 1) / 2) - math.lgamma(d / 2))
+    assert abs(np.linalg.norm(W, axis=1).mean() - chi_mean) < 0.02
+
+
+# ------------------------------------------------------------------ Monte-Carlo: unbiasedness, variance, M
+def _mc_estimates(q, k, M, n, kind, structured):
+    d = q.shape[1]
+    est = np.empty((n, q.shape[0], k.shape[0]))
+    for s in range(n):
+        if structured:
+            G, R = fi.orf_gaussians(1, M, d, seed=50000 + s)
+            om = O.orf_matrix(G[0], R[0], M)
+        else:
+            om = fi.iid_gaussians(1, M, d, seed=50000 + s)[0]
+        est[s] = O.phi(q, om, kind) @ O.phi(k, om, kind).T
+    return est
+
+
+def _arccos_kernel(q, k):
+    nq = np.linalg.norm(q, axis=1)[:, None]
+    nk = np.linalg.norm(k, axis=1)[None, :]
+    c = np.clip(q @ k.T / (nq * nk), -1, 1)
+    t = np.arccos(c)
+    return nq * nk * (np.sin(t) + (np.pi - t) * c) / (2 * np.pi)
+
+
+@pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
+@pytest.mark.parametrize("structured", [True, False])
+def test_kernel_estimate_is_unbiased(kind, structured):
+    q, k, _ = _qkv(16, 16, seed=21)
+    n = 3000
+    est = _mc_estimates(q, k[:12], 32, n, kind, structured)
+    exact = np.exp(q @ k[:12].T) if kind == O.TRIG else _arccos_kernel(q, k[:12])
+    z = (est.mean(axis=0) - exact) / (est.std(axis=0, ddof=1) / math.sqrt(n))
+    # the pairs share the same draws, so their z-scores are correlated: bound each one
+    assert np.abs(z).max() < 4.5
+
+
+def test_trig_variance_closed_form_and_orf_reduction():
+    # small |q - k|, where orthogonal directions cut the variance most
+    q, k, _ = _qkv(10, 16, seed=31)
+    q, k = 0.5 * q, 0.5 * k[:10]
+    n, M = 2000, 32
+    iid = _mc_estimates(q, k, M, n, O.TRIG, structured=False)
+    orf = _mc_estimates(q, k, M, n, O.TRIG, structured=True)
+    nq = np.sum(q * q, axis=1)[:, None]
+    nk = np.sum(k * k, axis=1)[None, :]
+    dd = np.sum((q[:, None, :] - k[None, :, :]) ** 2, axis=2)
+    closed = np.exp(nq + nk) * (1 - np.exp(-dd)) ** 2 / (2 * M)
+    ratio = iid.var(axis=0, ddof=1) / closed
+    assert 0.9 < ratio.mean() < 1.1
+    assert np.all((ratio > 0.75) & (ratio < 1.3))
+    assert (orf.var(axis=0, ddof=1) / closed).mean() < 0.5
+
+
+@pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
+def test_error_shrinks_with_feature_count(kind):
+    q, k, v = _qkv(64, 16, seed=41)
+    ref = (O.softmax_attention_head(q, k, v, False) if kind == O.TRIG
+           else O.arccos_attention_head(q, k, v, False))
+    Ms = [16, 64, 256, 1024]
+    err = []
+    for M in Ms:
+        e = []
+        for s in range(16):
+            G, R = fi.orf_gaussians(1, M, 16, seed=7000 + 97 * s + M)
+            om = O.orf_matrix(G[0], R[0], M)
+            e.append(np.median(np.abs(O.favor_bidirectional_head(q, k, v, om, kind) - ref)))
+        # medians: the trig ratio estimator has a signed denominator and heavy tails
+        err.append(np.median(e))
+    assert all(err[i + 1] < err[i] for i in range(len(err) - 1))
+    slope = np.polyfit(np.log(Ms), np.log(err), 1)[0]
+    assert -0.7 < slope < -0.35
