@@ -1,0 +1,318 @@
+#!/usr/bin/env python
+"""FAVOR forward benchmark: tokens/s (B*H*L per second) at B=4, H=8, L=4096, d=64, M=256.
+
+One step is one pass of the hot path over one batch: the trig and the ReLU feature maps, each
+bidirectional and causal, on the same bf16 inputs. value = head-tokens processed per second
+over all ranks (4 variants x B*H*L per step per rank). Inputs are resident in HBM. Four
+rotating input sets (268 MB in total, more than 2x the 126 MB L2) keep every step reading HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 is launched by torch.distributed.run. Each rank runs its own batch on its own GPU (the
+heads are independent), so per-GPU work is fixed ("weak" scaling) and there is no data-path
+collective. Timing: CUDA events on the launching stream, barrier + synchronize on both sides,
+max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(B=4, H=8, L=4096, d=64, M=256)
+VARIANTS = [("trig_bidir", 0, False), ("relu_bidir", 1, False)]
+N_SETS = 4
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "FAVOR fwd tokens/s (B·H·L/s) at L=4096,d=64,M=256; % of tensor/HBM roofline"
+
+
+def flops_per_token(d, M, kind):
+    F = 2 * M if kind == 0 else M
+    return 4 * d * M + 4 * F * (d + 1)
+
+
+def bytes_per_token(d):
+    return 4 * d * 2  # read q, k, v and write out, bf16
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples (SM clock, max clock, throttle reasons) while the timed region runs."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.rows, self.proc, self.t = index, [], None, None
+        self.active = threading.Event()
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "50",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+        time.sleep(0.5)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            if self.active.is_set():
+                self.rows.append([x.strip() for x in line.split(",")])
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm = []
+        mx = None
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[0]))
+                mx = float(r[1])
+                for n, val in zip(names, r[3:7]):
+                    if val.lower() == "active":
+                        reasons.add(n)
+            except Exception:
+                continue
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(seconds, per_step=False):
+    """Time the fp64 oracle (as it stands) on whole heads of the bench workload."""
+    import numpy as np
+
+    import favor_inputs as fi
+    from oracle import favor_oracle as O
+    W = WORKLOAD
+    q, k, v = fi.qkv(1, 1, W["L"], W["d"], seed=123)
+    G, R = fi.orf_gaussians(1, W["M"], W["d"], seed=123)
+    om = O.orf_matrices(G, R, W["M"])[0]
+    q, k, v = (x[0, 0].astype(np.float64) for x in (q, k, v))
+    tokens, t0, heads = 0, time.perf_counter(), 0
+    while True:
+        for _, kind, causal in VARIANTS:
+            (O.favor_causal_head if causal else O.favor_bidirectional_head)(q, k, v, om, kind)
+            tokens += W["L"]
+        heads += 1
+        if per_step or time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return tokens / dt, dt, heads
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(0, per_step=True)
+    tok, dt = 0.0, 0.0
+    for _ in range(args.steps):
+        r, t, _ = oracle_sample(0, per_step=True)
+        tok += r * t
+        dt += t
+    value = tok / dt
+    W = WORKLOAD
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / max(args.steps, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "favor_fwd_B4_H8_L4096_d64_M256", **W,
+                   "variants": [n for n, _, _ in VARIANTS]},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": "one head (L=4096 tokens) per variant per step, fp64 numpy oracle"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    args.warmup = max(args.warmup, 3)
+
+    import numpy as np
+    import torch
+
+    import favor_inputs as fi
+    import linear_kernelized_attention_b200 as F
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    W = WORKLOAD
+    B, H, L, d, M = W["B"], W["H"], W["L"], W["d"], W["M"]
+    stream = torch.cuda.current_stream()
+    variants = VARIANTS
+
+    # inputs: N_SETS rotating sets, Omega built on the device from seeded Gaussian draws
+    sets = []
+    for s in range(N_SETS):
+        q, k, v = fi.qkv(B, H, L, d, seed=1000 * rank + s)
+        sets.append([fi.round_to(x, "bf16").to(dev) for x in (q, k, v)])
+    G, R = fi.orf_gaussians(H, M, d, seed=rank)
+    omega = F.favor_orf_omega(torch.from_numpy(G).to(dev), torch.from_numpy(R).to(dev), M,
+                              dtype=torch.bfloat16)
+    outs = [[torch.empty_like(sets[0][0]) for _ in variants] for _ in range(N_SETS)]
+
+    def step(i, ev=None):
+        q, k, v = sets[i % N_SETS]
+        for j, (_, kind, causal) in enumerate(variants):
+            if ev is not None:
+                ev[j][0].record(stream)
+            F.favor_attention(q, k, v, omega, out=outs[i % N_SETS][j], feature_kind=kind, causal=causal,
+                              stream=stream)
+            if ev is not None:
+                ev[j][1].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if F.favor_sync_status(stream) != 0:
+        raise RuntimeError("device status not OK after warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+            for _ in variants] for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.active.set()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.active.clear()
+    if dist:
+        dist.barrier()
+    clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if F.favor_sync_status(stream) != 0:
+        raise RuntimeError("device status not OK after the timed region")
+    per_variant = {name: float(np.mean([evs[i][j][0].elapsed_time(evs[i][j][1]) for i in range(args.steps)]))
+                   for j, (name, _, _) in enumerate(variants)}
+    tokens_step = len(variants) * B * H * L
+    value = world * tokens_step / (ms * 1e-3)
+
+    # roofline of the dominant kernel (each variant is one kernel launch)
+    peaks, peak_src = load_peaks()
+    dom = max(per_variant, key=per_variant.get)
+    kind = [vv[1] for vv in variants if vv[0] == dom][0]
+    flops = flops_per_token(d, M, kind) * B * H * L
+    achieved = flops / (per_variant[dom] * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": None, "kernel": dom,
+            "peak_source": f"{peak_src} bf16 burst", "ms_per_launch": per_variant[dom]}
+
+    # end to end through the host-buffer C ABI entry (pinned host memory, copies timed)
+    e2e = None
+    hq, hk, hv = (x.cpu().pin_memory() for x in sets[0])
+    hom = omega.cpu().pin_memory()
+    hout = torch.empty_like(hq).pin_memory()
+    n_e2e = min(args.steps, 10)
+    for _, kind, causal in variants:
+        F.favor_attention_host(hq, hk, hv, hom, hout, feature_kind=kind, causal=causal)
+    if dist:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(n_e2e):
+        for _, kind, causal in variants:
+            F.favor_attention_host(hq, hk, hv, hom, hout, feature_kind=kind, causal=causal)
+    e2e_s = (time.perf_counter() - t0) / n_e2e
+    if dist:
+        t = torch.tensor([e2e_s], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    nx = B * H * L * d * 2
+    e2e = {"value": world * tokens_step / e2e_s, "unit": "tokens/s",
+           "h2d_bytes_per_step": len(variants) * (3 * nx + H * M * d * 2),
+           "d2h_bytes_per_step": len(variants) * nx}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r, dt, heads = oracle_sample(10.0)
+        cpu = {"value": r, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{heads} head(s) x L=4096 tokens x {len(VARIANTS)} variants, fp64 numpy, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "favor_fwd_B4_H8_L4096_d64_M256", **W,
+                       "variants": [vv[0] for vv in variants], "ms_per_launch": per_variant,
+                       "l2": f"{N_SETS} rotating input sets ({N_SETS * 4 * B * H * L * d * 2 / 1e6:.0f} MB) > 2x L2",
+                       "parallelism": f"replica x{world} (independent heads per rank)"},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps * len(variants), "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

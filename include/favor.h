@@ -1,0 +1,150 @@
+/*
+ * favor.h - C ABI of libfavor.so, the B200 (sm_100a) FAVOR attention forward pass.
+ *
+ * The operation. For each head h and batch b, with Q, K, V in R^{L x d} and Omega_h in R^{M x d}:
+ *   out = D_hat^-1 (phi(Q) (phi(K)^T [V | 1]))
+ * This is softmax attention D^-1 A V, A = exp(Q K^T / sqrt(d)), with the kernel factored as
+ * exp(q.k) ~ phi(q).phi(k). phi(K)^T [V|1] (an F x (d+1) state) is formed first, then
+ * left-multiplied by phi(Q), so no L x L matrix is formed. Source: the explainer page
+ * "用随机特征“骗”过 softmax，Transformer 注意力也能跑成线性？" (arXiv 2009.14794), section
+ * "核心机制：FAVOR+". The feature maps:
+ *   FAVOR_TRIG: phi(x) = exp(|x|^2/2)/sqrt(M) [cos(Omega x), sin(Omega x)], F = 2M.
+ *               The random Fourier features of the Gaussian kernel ("Masked Language
+ *               Modeling for Proteins via Linearly Scalable Long-Context Transformers",
+ *               Methodology / 方法详解).
+ *   FAVOR_RELU: phi(x) = max(Omega x, 0)/sqrt(M), F = M. A generalized-attention kernel
+ *               (the same paper, 核心创新).
+ * causal != 0 sums over keys j <= i only. This is the prefix sum of phi(k_j)[v_j|1]^T
+ * from the explainer's 核心机制 section.
+ *
+ * Scaling. The library computes exp(q.k) of q and k as passed. The 1/sqrt(d) temperature is
+ * the caller's d^-1/4 pre-scale of Q and K. Constant factors that cancel between numerator
+ * and denominator are dropped: 1/sqrt(M), exp(|q|^2/2), and a per-head max of |k|^2/2
+ * (the stabiliser). They do not change the result.
+ *
+ * Layout. Everything is row-major and contiguous:
+ *   q, k, v, out: [B, H, L, d], d contiguous.
+ *   omega:        [H, M, d], one matrix per head, shared across the batch.
+ *
+ * Ownership. Every pointer is owned by the caller. The library frees nothing and keeps no
+ * pointer after a call returns. Device pointers must be on the current device.
+ *
+ * Streams. Calls are asynchronous and ordered on `stream`, passed as a cudaStream_t
+ * (NULL means the legacy default stream). The return value reports argument validation and
+ * launch errors. Errors from inside a kernel surface at the next synchronisation.
+ * favor_sync_status() synchronises the stream and returns the device-side status word.
+ *
+ * Scratch. Calls that need scratch take it from cudaMallocAsync on `stream` and release it
+ * with cudaFreeAsync on the same stream.
+ *
+ * Errors. Negative favor_status codes. On an error nothing is launched and no output is
+ * written.
+ */
+#ifndef FAVOR_H_
+#define FAVOR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FAVOR_TRIG = 0, /* cos/sin softmax-kernel random features, F = 2M */
+  FAVOR_RELU = 1  /* ReLU generalized-attention features, F = M */
+} favor_feature_kind;
+
+typedef enum {
+  FAVOR_OK = 0,
+  FAVOR_ERR_NULL = -1,        /* a required pointer is NULL */
+  FAVOR_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned */
+  FAVOR_ERR_SHAPE = -3,       /* a size is non-positive or the total overflows */
+  FAVOR_ERR_KIND = -4,        /* feature_kind is not FAVOR_TRIG / FAVOR_RELU */
+  FAVOR_ERR_UNSUPPORTED = -5, /* a valid shape this build has no kernel for */
+  FAVOR_ERR_CUDA = -6,        /* a CUDA runtime call failed (launch, allocation, copy) */
+  FAVOR_ERR_TIMEOUT = -7,     /* a bounded device-side wait gave up */
+  FAVOR_ERR_DEVICE = -8       /* the current device is not sm_100 */
+} favor_status;
+
+/*
+ * bf16 forward pass: the tensor-core path.
+ * q, k, v, omega, out: device pointers to __nv_bfloat16, 16-byte aligned, layouts above.
+ * Supported: d in {32, 64}; M a multiple of 16 with 16 <= M <= 256 (trig) or <= 512 (relu);
+ * L >= 1 (ragged tails are masked); B*H <= 65535.
+ * Arithmetic: Q Omega^T and K Omega^T on tensor cores (bf16 in, fp32 accumulate).
+ * Features in fp32 registers. phi(K) is rounded to bf16 for phi(K)^T [V|1] (fp32 accumulate).
+ * The state is rounded to fp16 under a power-of-two scale, phi(Q) to fp16, and
+ * phi(Q) S is accumulated in fp32. The normaliser division is in fp32, and the result is
+ * rounded once to bf16.
+ * A zero denominator gives a zero output row.
+ */
+int favor_attention(const void* q, const void* k, const void* v, const void* omega, void* out,
+                    int B, int H, int L, int d, int M, int feature_kind, int causal,
+                    void* stream);
+
+/*
+ * As favor_attention, with an explicit causal chunk length (64 or 128 tokens; 0 picks
+ * the default). The chunk changes how the prefix sum is blocked, not its value.
+ * Ignored when causal == 0.
+ */
+int favor_attention_chunked(const void* q, const void* k, const void* v, const void* omega,
+                            void* out, int B, int H, int L, int d, int M, int feature_kind,
+                            int causal, int chunk, void* stream);
+
+/*
+ * fp32 forward pass: the accuracy path (CUDA cores, fp32 throughout, accurate sin/cos/exp).
+ * q, k, v, omega, out: device pointers to float, 16-byte aligned, same layouts.
+ * Supported: 1 <= d <= 128, 1 <= M <= 512, L >= 1.
+ */
+int favor_attention_f32(const float* q, const float* k, const float* v, const float* omega,
+                        float* out, int B, int H, int L, int d, int M, int feature_kind,
+                        int causal, void* stream);
+
+/*
+ * Orthogonal random features (ORF) Omega, built on the device from Gaussian draws.
+ * "Masked Language Modeling for Proteins via Linearly Scalable Long-Context Transformers"
+ * (方法详解; 实验设计 ablation) and the explainer's 核心机制 section: random directions
+ * constrained to a random subsample of an orthogonal matrix.
+ *   gauss_blocks: device double [H, ceil(M/d), d, d], i.i.d. N(0,1). Each d x d block's rows
+ *                 are orthonormalised in order (Gram-Schmidt, fp64).
+ *   gauss_norms:  device double [H, M, d], i.i.d. N(0,1). Row r of Omega_h is scaled by
+ *                 |gauss_norms[h, r, :]|, a chi_d length.
+ *   omega:        device output [H, M, d], dtype per omega_dtype (0 = float, 1 = bf16).
+ * Blocks are stacked and cut to M rows. Supported: 1 <= d <= 128, 1 <= M.
+ */
+int favor_orf_omega(const double* gauss_blocks, const double* gauss_norms, void* omega,
+                    int H, int M, int d, int omega_dtype, void* stream);
+
+/*
+ * Host-buffer convenience entry: q, k, v, omega, out are HOST pointers (pinned memory
+ * makes the copies asynchronous). Allocates device buffers with cudaMallocAsync on
+ * `stream`, copies in, runs favor_attention (dtype_code 1 = bf16) or favor_attention_f32
+ * (dtype_code 0 = float), copies out and frees. It synchronises `stream` before returning,
+ * so `out` is ready when it returns FAVOR_OK.
+ */
+int favor_attention_host(const void* q, const void* k, const void* v, const void* omega,
+                         void* out, int B, int H, int L, int d, int M, int feature_kind,
+                         int causal, int dtype_code, void* stream);
+
+/* Synchronise `stream`, then read and clear the device status word (FAVOR_OK or a code). */
+int favor_sync_status(void* stream);
+
+/* Static description of a status code. Never NULL. */
+const char* favor_status_string(int status);
+
+/*
+ * Self-test of the bounded device-side waits (no counterpart on the pages). Launches one block
+ * that waits on a barrier nothing completes, for at most `limit_cycles` SM clock cycles
+ * (0 < limit_cycles <= 4e9). favor_sync_status() afterwards returns FAVOR_ERR_TIMEOUT, and the
+ * context stays usable.
+ */
+int favor_selftest_timeout(long long limit_cycles, void* stream);
+
+/* Bytes of scratch one favor_attention call takes from cudaMallocAsync (0 if none). */
+size_t favor_workspace_bytes(int B, int H, int L, int d, int M, int feature_kind, int causal);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FAVOR_H_ */

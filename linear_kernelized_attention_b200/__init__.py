@@ -1,0 +1,174 @@
+"""B200 (sm_100a) FAVOR attention forward pass: Python binding of libfavor.so.
+
+The binding only marshals arguments. Every step of the computation runs in the CUDA kernels
+of ``libfavor.so``, and PyTorch supplies device memory and streams. There is no CPU fallback:
+if the library is missing or a call fails, an exception is raised.
+
+Entry points mirror the C ABI in include/favor.h:
+    favor_attention, favor_attention_chunked, favor_attention_f32, favor_orf_omega,
+    favor_attention_host, favor_sync_status, favor_status_string, favor_workspace_bytes,
+    favor_selftest_timeout
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+FAVOR_TRIG = 0
+FAVOR_RELU = 1
+STATUS = {
+    0: "FAVOR_OK", -1: "FAVOR_ERR_NULL", -2: "FAVOR_ERR_ALIGN", -3: "FAVOR_ERR_SHAPE",
+    -4: "FAVOR_ERR_KIND", -5: "FAVOR_ERR_UNSUPPORTED", -6: "FAVOR_ERR_CUDA",
+    -7: "FAVOR_ERR_TIMEOUT", -8: "FAVOR_ERR_DEVICE",
+}
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfavor.so")
+
+_vp, _i, _ll, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t
+_SIGS = {
+    "favor_attention": (_i, [_vp] * 5 + [_i] * 7 + [_vp]),
+    "favor_attention_chunked": (_i, [_vp] * 5 + [_i] * 8 + [_vp]),
+    "favor_attention_f32": (_i, [_vp] * 5 + [_i] * 7 + [_vp]),
+    "favor_orf_omega": (_i, [_vp] * 3 + [_i] * 4 + [_vp]),
+    "favor_attention_host": (_i, [_vp] * 5 + [_i] * 8 + [_vp]),
+    "favor_sync_status": (_i, [_vp]),
+    "favor_status_string": (ctypes.c_char_p, [_i]),
+    "favor_selftest_timeout": (_i, [_ll, _vp]),
+    "favor_workspace_bytes": (_sz, [_i] * 7),
+}
+_LIB = None
+
+
+class FavorError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({favor_status_string(code)})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfavor.so (built in-tree). Raises ImportError if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; build it with "
+                              "`python -m linear_kernelized_attention_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _LIB = L
+    return _LIB
+
+
+def favor_status_string(code: int) -> str:
+    return lib().favor_status_string(int(code)).decode()
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise FavorError(rc, where)
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_qkv(q, k, v, omega, dtype):
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v), ("omega", omega)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+        if t.dtype != dtype:
+            raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share the shape [B, H, L, d]")
+    B, H, L, d = q.shape
+    if omega.dim() != 3 or omega.shape[0] != H or omega.shape[2] != d:
+        raise ValueError("omega must have shape [H, M, d]")
+    return B, H, L, d, omega.shape[1]
+
+
+def favor_attention(q, k, v, omega, out=None, feature_kind=FAVOR_TRIG, causal=False, chunk=0,
+                    stream=None):
+    """bf16 FAVOR forward on the tensor-core path. q, k, v: [B,H,L,d]; omega: [H,M,d]."""
+    import torch
+    B, H, L, d, M = _check_qkv(q, k, v, omega, torch.bfloat16)
+    if out is None:
+        out = torch.empty_like(q)
+    rc = lib().favor_attention_chunked(q.data_ptr(), k.data_ptr(), v.data_ptr(), omega.data_ptr(),
+                                       out.data_ptr(), B, H, L, d, M, int(feature_kind), int(causal),
+                                       int(chunk), _stream(stream))
+    _check(rc, "favor_attention")
+    return out
+
+
+def favor_attention_chunked(q, k, v, omega, out=None, feature_kind=FAVOR_TRIG, causal=False,
+                            chunk=0, stream=None):
+    return favor_attention(q, k, v, omega, out, feature_kind, causal, chunk, stream)
+
+
+def favor_attention_f32(q, k, v, omega, out=None, feature_kind=FAVOR_TRIG, causal=False,
+                        stream=None):
+    """fp32 FAVOR forward on the accuracy path."""
+    import torch
+    B, H, L, d, M = _check_qkv(q, k, v, omega, torch.float32)
+    if out is None:
+        out = torch.empty_like(q)
+    rc = lib().favor_attention_f32(q.data_ptr(), k.data_ptr(), v.data_ptr(), omega.data_ptr(),
+                                   out.data_ptr(), B, H, L, d, M, int(feature_kind), int(causal),
+                                   _stream(stream))
+    _check(rc, "favor_attention_f32")
+    return out
+
+
+def favor_orf_omega(gauss_blocks, gauss_norms, M, dtype=None, out=None, stream=None):
+    """Build ORF Omega [H, M, d] on the device from fp64 Gaussian draws (see include/favor.h)."""
+    import torch
+    dtype = dtype or torch.bfloat16
+    H, nb, d, d2 = gauss_blocks.shape
+    if d != d2 or gauss_norms.shape != (H, M, d) or nb != -(-M // d):
+        raise ValueError("gauss_blocks must be [H, ceil(M/d), d, d] and gauss_norms [H, M, d]")
+    for t in (gauss_blocks, gauss_norms):
+        if t.dtype != torch.float64 or not t.is_cuda or not t.is_contiguous():
+            raise TypeError("Gaussian draws must be contiguous float64 CUDA tensors")
+    if out is None:
+        out = torch.empty((H, M, d), dtype=dtype, device=gauss_blocks.device)
+    code = {torch.float32: 0, torch.bfloat16: 1}[out.dtype]
+    rc = lib().favor_orf_omega(gauss_blocks.data_ptr(), gauss_norms.data_ptr(), out.data_ptr(), H, M,
+                               d, code, _stream(stream))
+    _check(rc, "favor_orf_omega")
+    return out
+
+
+def favor_attention_host(q, k, v, omega, out, feature_kind=FAVOR_TRIG, causal=False, stream=None):
+    """Host-buffer entry: q, k, v, omega, out are CPU tensors (pinned for async copies)."""
+    import torch
+    for t in (q, k, v, omega, out):
+        if t.is_cuda or not t.is_contiguous():
+            raise TypeError("favor_attention_host takes contiguous CPU tensors")
+    code = {torch.float32: 0, torch.bfloat16: 1}[q.dtype]
+    B, H, L, d = q.shape
+    M = omega.shape[1]
+    rc = lib().favor_attention_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), omega.data_ptr(),
+                                    out.data_ptr(), B, H, L, d, M, int(feature_kind), int(causal),
+                                    code, _stream(stream))
+    _check(rc, "favor_attention_host")
+    return out
+
+
+def favor_sync_status(stream=None) -> int:
+    return lib().favor_sync_status(_stream(stream))
+
+
+def favor_workspace_bytes(B, H, L, d, M, feature_kind=FAVOR_TRIG, causal=False) -> int:
+    return lib().favor_workspace_bytes(B, H, L, d, M, int(feature_kind), int(causal))
+
+
+def favor_selftest_timeout(limit_cycles: int, stream=None) -> int:
+    return lib().favor_selftest_timeout(int(limit_cycles), _stream(stream))

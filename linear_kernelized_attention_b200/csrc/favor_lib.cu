@@ -1,0 +1,394 @@
+// favor_lib.cu - host side of libfavor.so: argument validation, TMA descriptors, scratch,
+// launches and the C ABI declared in include/favor.h. All device code is included here, so
+// the library is one translation unit with one device status word.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/favor.h"
+#include "ptx.cuh"
+#include "kernels_f32.cuh"
+#include "kernel_bidir.cuh"
+
+namespace favor {
+
+// A kernel whose only job is a bounded wait on an mbarrier nobody arrives on. It checks that
+// the timeout path records FAVOR_ERR_TIMEOUT and returns, leaving the context usable.
+__global__ void k_selftest_timeout(long long limit_cycles) {
+  __shared__ uint64_t b;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&b), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  mbar_wait(smem_u32(&b), 0, nullptr, limit_cycles);
+  __syncthreads();
+}
+}  // namespace favor
+
+namespace {
+
+using namespace favor;
+
+#define FAVOR_TRY(expr)                          \
+  do {                                           \
+    if ((expr) != cudaSuccess) return FAVOR_ERR_CUDA; \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FAVOR_ERR_CUDA;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return FAVOR_ERR_CUDA;
+  return major == 10 ? FAVOR_OK : FAVOR_ERR_DEVICE;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+// Common shape/pointer checks shared by every entry point.
+int check_common(const void* q, const void* k, const void* v, const void* omega, const void* out,
+                 int B, int H, int L, int d, int M, int kind) {
+  if (!q || !k || !v || !omega || !out) return FAVOR_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(omega) || !aligned16(out))
+    return FAVOR_ERR_ALIGN;
+  if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || M <= 0) return FAVOR_ERR_SHAPE;
+  if ((long long)B * H > INT_MAX / 2 || (long long)B * H * L > (1ll << 40) ||
+      (long long)B * H * L * d > (1ll << 40))
+    return FAVOR_ERR_SHAPE;
+  if (kind != FAVOR_TRIG && kind != FAVOR_RELU) return FAVOR_ERR_KIND;
+  return FAVOR_OK;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor [n2][n1][64] with 128-byte rows, box {64, 128, 1}, 128-byte swizzle,
+// out-of-range rows read as zero and are not written.
+bool make_map_rows64(CUtensorMap* m, const void* ptr, uint64_t n1, uint64_t n2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {64, n1, n2};
+  const cuuint64_t strides[2] = {128, 128 * n1};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ scratch
+// Scratch comes from a library-owned stream-ordered pool (per device) that keeps its memory
+// between calls, so repeated calls do not return memory to the driver.
+cudaMemPool_t pool_for_device() {
+  static cudaMemPool_t pools[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> g(mu);
+  if (dev < 0 || dev >= 64) return nullptr;
+  if (!pools[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    if (cudaMemPoolCreate(&pools[dev], &props) != cudaSuccess) return nullptr;
+    uint64_t thr = UINT64_MAX;
+    cudaMemPoolSetAttribute(pools[dev], cudaMemPoolAttrReleaseThreshold, &thr);
+  }
+  return pools[dev];
+}
+
+int scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
+  *p = nullptr;
+  if (bytes == 0) return FAVOR_OK;
+  cudaMemPool_t pool = pool_for_device();
+  if (!pool) return FAVOR_ERR_CUDA;
+  return cudaMallocFromPoolAsync(p, bytes, pool, st) == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ bf16 bidirectional plan
+struct BidirPlan {
+  int P, Mpad, nsb, Fpad, natoms, ntiles;
+  size_t part_bytes, meta_bytes, image_bytes;
+};
+
+BidirPlan plan_bidir(int BH, int L, int M, int kind) {
+  BidirPlan pl{};
+  pl.Mpad = (M + 127) / 128 * 128;
+  pl.nsb = kind == FAVOR_TRIG ? 2 * pl.Mpad / 128 : pl.Mpad / 128;
+  pl.Fpad = pl.nsb * 128;
+  pl.natoms = pl.Fpad / 64;
+  pl.ntiles = (L + tc::kTile - 1) / tc::kTile;
+  int P = sm_count() / BH;
+  if (P < 1) P = 1;
+  if (P > 8) P = 8;
+  if (P > pl.ntiles) P = pl.ntiles;
+  pl.P = P;
+  if (P > 1) {
+    pl.part_bytes = (size_t)BH * P * tc::kNV * pl.Fpad * sizeof(float);
+    pl.meta_bytes = ((size_t)BH * P * 2 * sizeof(float) + 255) / 256 * 256;
+    pl.image_bytes = (size_t)BH * pl.natoms * tc::kImgAtomB;
+  }
+  return pl;
+}
+
+int check_tc_shape(int d, int M, int kind) {
+  if (d != 64) return FAVOR_ERR_UNSUPPORTED;
+  if (M % 16 != 0) return FAVOR_ERR_UNSUPPORTED;
+  if (kind == FAVOR_TRIG && M > 256) return FAVOR_ERR_UNSUPPORTED;
+  if (kind == FAVOR_RELU && M > 512) return FAVOR_ERR_UNSUPPORTED;
+  return FAVOR_OK;
+}
+
+int launch_bidir_bf16(const void* q, const void* k, const void* v, const void* omega, void* out,
+                      int B, int H, int L, int M, int kind, cudaStream_t st) {
+  const int BH = B * H;
+  if (BH > 65535 * 8) return FAVOR_ERR_UNSUPPORTED;
+  const BidirPlan pl = plan_bidir(BH, L, M, kind);
+  CUtensorMap mq, mk, mv, mo, mom;
+  if (!make_map_rows64(&mq, q, L, BH) || !make_map_rows64(&mk, k, L, BH) ||
+      !make_map_rows64(&mv, v, L, BH) || !make_map_rows64(&mo, out, L, BH) ||
+      !make_map_rows64(&mom, omega, M, H))
+    return FAVOR_ERR_CUDA;
+  void* ws = nullptr;
+  const size_t ws_bytes = pl.part_bytes + pl.meta_bytes + pl.image_bytes;
+  int rc = scratch_alloc(&ws, ws_bytes, st);
+  if (rc != FAVOR_OK) return rc;
+  tc::BidirParams prm{};
+  prm.BH = BH;
+  prm.H = H;
+  prm.L = L;
+  prm.M = M;
+  prm.Mpad = pl.Mpad;
+  prm.P = pl.P;
+  prm.ntiles = pl.ntiles;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  prm.part = reinterpret_cast<float*>(w);
+  prm.pmeta = reinterpret_cast<float*>(w + pl.part_bytes);
+  prm.image = w + pl.part_bytes + pl.meta_bytes;
+  const uint32_t smem = tc::bidir_smem_bytes(pl.Mpad);
+  auto kern = kind == FAVOR_TRIG ? tc::favor_bidir_tc<0> : tc::favor_bidir_tc<1>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    rc = FAVOR_ERR_CUDA;
+  if (rc == FAVOR_OK) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(BH * pl.P, 1, 1);
+    cfg.blockDim = dim3(tc::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.P;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mom, mo, prm) != cudaSuccess) rc = FAVOR_ERR_CUDA;
+  }
+  if (ws) cudaFreeAsync(ws, st);
+  return rc;
+}
+
+// ------------------------------------------------------------------ fp32 path
+size_t f32_workspace(int BH, int L, int d, int M, int kind) {
+  const int F = kind == FAVOR_TRIG ? 2 * M : M;
+  const int nch = (L + f32::kChunk - 1) / f32::kChunk;
+  return (size_t)BH * nch * F * (d + 1) * sizeof(float) + (size_t)BH * sizeof(float);
+}
+
+int launch_f32(const float* q, const float* k, const float* v, const float* omega, float* out,
+               int B, int H, int L, int d, int M, int kind, int causal, cudaStream_t st) {
+  const int BH = B * H;
+  const int F = kind == FAVOR_TRIG ? 2 * M : M;
+  const int nch = (L + f32::kChunk - 1) / f32::kChunk;
+  const int nft = (F + f32::kFeatTile - 1) / f32::kFeatTile;
+  if (BH > 65535 || nch > 65535) return FAVOR_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  int rc = scratch_alloc(&ws, f32_workspace(BH, L, d, M, kind), st);
+  if (rc != FAVOR_OK) return rc;
+  float* dS = static_cast<float*>(ws);
+  float* cmax = dS + (size_t)BH * nch * F * (d + 1);
+  const size_t sm_state = (size_t)(2 * f32::kChunk * d + f32::kChunk + f32::kChunk * f32::kFeatTile) * 4;
+  const size_t sm_out = (size_t)(3 * f32::kChunk * d + f32::kChunk + 2 * f32::kChunk * f32::kFeatTile +
+                                 f32::kFeatTile * (d + 1) + f32::kChunk * f32::kChunk) * 4;
+  if (cudaFuncSetAttribute(f32::k_chunk_state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_state) != cudaSuccess ||
+      cudaFuncSetAttribute(f32::k_output, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out) != cudaSuccess)
+    rc = FAVOR_ERR_CUDA;
+  if (rc == FAVOR_OK) {
+    if (kind == FAVOR_TRIG) f32::k_key_halfnorm_max<<<BH, f32::kThreads, 0, st>>>(k, cmax, L, d);
+    f32::k_chunk_state<<<dim3(nft, nch, BH), f32::kThreads, sm_state, st>>>(k, v, omega, cmax, dS, H, L,
+                                                                             d, M, F, kind);
+    const long long per_chunk = (long long)F * (d + 1);
+    const long long total = (long long)BH * per_chunk;
+    f32::k_scan_chunks<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(dS, nch, per_chunk, total, causal);
+    f32::k_output<<<dim3(nch, BH), f32::kThreads, sm_out, st>>>(q, k, v, omega, cmax, dS, out, H, L, d, M,
+                                                                F, kind, causal);
+    if (cudaGetLastError() != cudaSuccess) rc = FAVOR_ERR_CUDA;
+  }
+  cudaFreeAsync(ws, st);
+  return rc;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* favor_status_string(int status) {
+  switch (status) {
+    case FAVOR_OK: return "ok";
+    case FAVOR_ERR_NULL: return "a required pointer is NULL";
+    case FAVOR_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case FAVOR_ERR_SHAPE: return "a size is non-positive or too large";
+    case FAVOR_ERR_KIND: return "feature_kind must be FAVOR_TRIG (0) or FAVOR_RELU (1)";
+    case FAVOR_ERR_UNSUPPORTED: return "shape not supported by this build";
+    case FAVOR_ERR_CUDA: return "a CUDA runtime call failed";
+    case FAVOR_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+    case FAVOR_ERR_DEVICE: return "the current device is not sm_100";
+    default: return "unknown favor status";
+  }
+}
+
+int favor_sync_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FAVOR_ERR_CUDA;
+  int s = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&s, favor::g_status, sizeof(int)) != cudaSuccess) return FAVOR_ERR_CUDA;
+  if (cudaMemcpyToSymbol(favor::g_status, &zero, sizeof(int)) != cudaSuccess) return FAVOR_ERR_CUDA;
+  return s;
+}
+
+size_t favor_workspace_bytes(int B, int H, int L, int d, int M, int feature_kind, int causal) {
+  if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || M <= 0) return 0;
+  (void)d;
+  (void)causal;
+  const BidirPlan pl = plan_bidir(B * H, L, M, feature_kind);
+  return pl.part_bytes + pl.meta_bytes + pl.image_bytes;
+}
+
+int favor_attention_chunked(const void* q, const void* k, const void* v, const void* omega,
+                            void* out, int B, int H, int L, int d, int M, int feature_kind,
+                            int causal, int chunk, void* stream) {
+  int rc = check_common(q, k, v, omega, out, B, H, L, d, M, feature_kind);
+  if (rc != FAVOR_OK) return rc;
+  if ((rc = check_device()) != FAVOR_OK) return rc;
+  if ((rc = check_tc_shape(d, M, feature_kind)) != FAVOR_OK) return rc;
+  if (chunk != 0 && chunk != 64 && chunk != 128) return FAVOR_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (causal) return FAVOR_ERR_UNSUPPORTED;
+  return launch_bidir_bf16(q, k, v, omega, out, B, H, L, M, feature_kind, st);
+}
+
+int favor_attention(const void* q, const void* k, const void* v, const void* omega, void* out,
+                    int B, int H, int L, int d, int M, int feature_kind, int causal, void* stream) {
+  return favor_attention_chunked(q, k, v, omega, out, B, H, L, d, M, feature_kind, causal, 0, stream);
+}
+
+int favor_attention_f32(const float* q, const float* k, const float* v, const float* omega,
+                        float* out, int B, int H, int L, int d, int M, int feature_kind,
+                        int causal, void* stream) {
+  int rc = check_common(q, k, v, omega, out, B, H, L, d, M, feature_kind);
+  if (rc != FAVOR_OK) return rc;
+  if ((rc = check_device()) != FAVOR_OK) return rc;
+  if (d > f32::kMaxD || M > 512) return FAVOR_ERR_UNSUPPORTED;
+  return launch_f32(q, k, v, omega, out, B, H, L, d, M, feature_kind, causal,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int favor_orf_omega(const double* gauss_blocks, const double* gauss_norms, void* omega, int H, int M,
+                    int d, int omega_dtype, void* stream) {
+  if (!gauss_blocks || !gauss_norms || !omega) return FAVOR_ERR_NULL;
+  if (!aligned16(gauss_blocks) || !aligned16(gauss_norms) || !aligned16(omega)) return FAVOR_ERR_ALIGN;
+  if (H <= 0 || M <= 0 || d <= 0) return FAVOR_ERR_SHAPE;
+  if (d > 128 || H > 65535) return FAVOR_ERR_UNSUPPORTED;
+  if (omega_dtype != 0 && omega_dtype != 1) return FAVOR_ERR_UNSUPPORTED;
+  int rc = check_device();
+  if (rc != FAVOR_OK) return rc;
+  const int nb = (M + d - 1) / d;
+  const size_t smem = (size_t)d * d * sizeof(double);
+  if (cudaFuncSetAttribute(k_orf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return FAVOR_ERR_CUDA;
+  k_orf<<<dim3(nb, H), 256, smem, static_cast<cudaStream_t>(stream)>>>(gauss_blocks, gauss_norms, omega, H,
+                                                                        M, d, omega_dtype);
+  return cudaGetLastError() == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
+}
+
+int favor_attention_host(const void* q, const void* k, const void* v, const void* omega, void* out,
+                         int B, int H, int L, int d, int M, int feature_kind, int causal,
+                         int dtype_code, void* stream) {
+  int rc = check_common(q, k, v, omega, out, B, H, L, d, M, feature_kind);
+  if (rc != FAVOR_OK) return rc;
+  if (dtype_code != 0 && dtype_code != 1) return FAVOR_ERR_UNSUPPORTED;
+  if ((rc = check_device()) != FAVOR_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t es = dtype_code == 1 ? 2 : 4;
+  const size_t nx = (size_t)B * H * L * d * es, nom = (size_t)H * M * d * es;
+  void *dq = nullptr, *dk = nullptr, *dv = nullptr, *dom = nullptr, *dout = nullptr;
+  if ((rc = scratch_alloc(&dq, nx, st)) != FAVOR_OK) return rc;
+  scratch_alloc(&dk, nx, st);
+  scratch_alloc(&dv, nx, st);
+  scratch_alloc(&dom, nom, st);
+  scratch_alloc(&dout, nx, st);
+  if (!dk || !dv || !dom || !dout) rc = FAVOR_ERR_CUDA;
+  if (rc == FAVOR_OK) {
+    if (cudaMemcpyAsync(dq, q, nx, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dk, k, nx, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dv, v, nx, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dom, omega, nom, cudaMemcpyHostToDevice, st) != cudaSuccess)
+      rc = FAVOR_ERR_CUDA;
+  }
+  if (rc == FAVOR_OK) {
+    rc = dtype_code == 1
+             ? favor_attention(dq, dk, dv, dom, dout, B, H, L, d, M, feature_kind, causal, stream)
+             : favor_attention_f32(static_cast<float*>(dq), static_cast<float*>(dk), static_cast<float*>(dv),
+                                   static_cast<float*>(dom), static_cast<float*>(dout), B, H, L, d, M,
+                                   feature_kind, causal, stream);
+  }
+  if (rc == FAVOR_OK && cudaMemcpyAsync(out, dout, nx, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    rc = FAVOR_ERR_CUDA;
+  for (void* p : {dq, dk, dv, dom, dout})
+    if (p) cudaFreeAsync(p, st);
+  if (cudaStreamSynchronize(st) != cudaSuccess && rc == FAVOR_OK) rc = FAVOR_ERR_CUDA;
+  return rc;
+}
+
+// Launch the bounded-wait self-test: a wait that nothing satisfies, limited to `limit_cycles`.
+// favor_sync_status() afterwards must report FAVOR_ERR_TIMEOUT.
+int favor_selftest_timeout(long long limit_cycles, void* stream) {
+  int rc = check_device();
+  if (rc != FAVOR_OK) return rc;
+  if (limit_cycles <= 0 || limit_cycles > 4000000000ll) return FAVOR_ERR_SHAPE;
+  favor::k_selftest_timeout<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles);
+  return cudaGetLastError() == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
+}
+
+}  // extern "C"

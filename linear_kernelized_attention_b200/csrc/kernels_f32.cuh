@@ -1,0 +1,320 @@
+// kernels_f32.cuh - fp32 FAVOR forward on CUDA cores (the accuracy path), plus the ORF builder.
+//
+// The arithmetic follows the explainer page "用随机特征“骗”过 softmax，Transformer 注意力也能跑成线性？",
+// section 核心机制：FAVOR+:
+//   - features phi(x) (cos/sin random features or ReLU generalized-attention features);
+//   - chunk states dS_c = sum_{j in chunk c} phi(k_j) [v_j | 1]^T;
+//   - a scan over chunks: exclusive prefix for causal, total for bidirectional;
+//   - out_i = (phi(q_i) S_i)[:d] / (phi(q_i) S_i)[d].
+//     Causal: S_i = (prefix before the chunk) + sum_{j in chunk, j <= i} phi(k_j)[v_j|1]^T.
+// Cancelling factors: 1/sqrt(M) and exp(|q|^2/2) are dropped, and the key factor is
+// exp(|k|^2/2 - c_h) with c_h = max_j |k_j|^2/2 of the head.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace favor {
+namespace f32 {
+
+constexpr int kChunk = 64;   // tokens per chunk
+constexpr int kFeatTile = 32;  // features per tile
+constexpr int kThreads = 256;
+constexpr int kMaxD = 128;
+
+// Feature f of token x (length d) with projection u = omega_a . x:
+//   trig: f <  M -> w cos(u_f),  f >= M -> w sin(u_{f-M})
+//   relu: max(u_f, 0)
+__device__ __forceinline__ float feature_value(int kind, int M, int f, const float* x,
+                                              const float* __restrict__ omega, int d, float w) {
+  const int a = (kind == 0 && f >= M) ? f - M : f;
+  const float* om = omega + (size_t)a * d;
+  float u = 0.f;
+  for (int t = 0; t < d; ++t) u = fmaf(om[t], x[t], u);
+  if (kind == 0) {
+    float s, c;
+    sincosf(u, &s, &c);
+    return w * (f < M ? c : s);
+  }
+  return fmaxf(u, 0.f);
+}
+
+// c_h = max_j |k_j|^2 / 2 for each head (trig stabiliser).
+__global__ void __launch_bounds__(kThreads) k_key_halfnorm_max(const float* __restrict__ k,
+                                                                float* __restrict__ cmax, int L,
+                                                                int d) {
+  const int bh = blockIdx.x;
+  const float* kh = k + (size_t)bh * L * d;
+  float m = -INFINITY;
+  for (int j = threadIdx.x; j < L; j += blockDim.x) {
+    float s = 0.f;
+    for (int t = 0; t < d; ++t) s = fmaf(kh[(size_t)j * d + t], kh[(size_t)j * d + t], s);
+    m = fmaxf(m, 0.5f * s);
+  }
+  __shared__ float red[kThreads / 32];
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float r = red[0];
+    for (int i = 1; i < kThreads / 32; ++i) r = fmaxf(r, red[i]);
+    cmax[bh] = r;
+  }
+}
+
+// dS[bh][c][f][n] = sum_{j in chunk c} phi_f(k_j) vv_j[n], vv_j = [v_j | 1], for one tile of
+// kFeatTile features. grid = (nfeat_tiles, nchunks, BH).
+__global__ void __launch_bounds__(kThreads)
+    k_chunk_state(const float* __restrict__ k, const float* __restrict__ v,
+                  const float* __restrict__ omega, const float* __restrict__ cmax,
+                  float* __restrict__ dS, int H, int L, int d, int M, int F, int kind) {
+  extern __shared__ float sm[];
+  float* sk = sm;                             // [kChunk][d]
+  float* sv = sk + kChunk * d;                // [kChunk][d]
+  float* sw = sv + kChunk * d;                // [kChunk]
+  float* sphi = sw + kChunk;                  // [kChunk][kFeatTile]
+  const int ft = blockIdx.x, c = blockIdx.y, bh = blockIdx.z, h = bh % H;
+  const int j0 = c * kChunk, nj = min(kChunk, L - j0);
+  const float* kh = k + ((size_t)bh * L + j0) * d;
+  const float* vh = v + ((size_t)bh * L + j0) * d;
+  const float* om = omega + (size_t)h * M * d;
+  for (int i = threadIdx.x; i < kChunk * d; i += blockDim.x) {
+    const bool ok = i < nj * d;
+    sk[i] = ok ? kh[i] : 0.f;
+    sv[i] = ok ? vh[i] : 0.f;
+  }
+  __syncthreads();
+  if (threadIdx.x < kChunk) {
+    const int j = threadIdx.x;
+    float w = 0.f;
+    if (j < nj) {
+      if (kind == 0) {
+        float s = 0.f;
+        for (int t = 0; t < d; ++t) s = fmaf(sk[j * d + t], sk[j * d + t], s);
+        w = expf(0.5f * s - cmax[bh]);
+      } else {
+        w = 1.f;
+      }
+    }
+    sw[j] = w;
+  }
+  __syncthreads();
+  for (int p = threadIdx.x; p < kChunk * kFeatTile; p += blockDim.x) {
+    const int j = p / kFeatTile, fl = p % kFeatTile, f = ft * kFeatTile + fl;
+    float val = 0.f;
+    if (j < nj && f < F) val = feature_value(kind, M, f, sk + j * d, om, d, sw[j]);
+    sphi[j * kFeatTile + fl] = (j < nj) ? val : 0.f;
+  }
+  __syncthreads();
+  const int dv = d + 1;
+  float* out = dS + (((size_t)bh * gridDim.y + c) * F) * dv;
+  for (int p = threadIdx.x; p < kFeatTile * dv; p += blockDim.x) {
+    const int fl = p / dv, n = p % dv, f = ft * kFeatTile + fl;
+    if (f >= F) continue;
+    float acc = 0.f;
+    for (int j = 0; j < nj; ++j) acc = fmaf(sphi[j * kFeatTile + fl], n < d ? sv[j * d + n] : 1.f, acc);
+    out[(size_t)f * dv + n] = acc;
+  }
+}
+
+// In-place scan over chunks for every (bh, f, n): exclusive prefix (causal) or the total,
+// written into chunk 0 (bidirectional).
+__global__ void k_scan_chunks(float* __restrict__ dS, int nchunks, long long per_chunk, long long total,
+                              int causal) {
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= total) return;
+  const long long bh = e / per_chunk, r = e % per_chunk;
+  float* p = dS + bh * nchunks * per_chunk + r;
+  float run = 0.f;
+  for (int c = 0; c < nchunks; ++c) {
+    const float x = p[c * per_chunk];
+    if (causal) p[c * per_chunk] = run;
+    run += x;
+  }
+  if (!causal) p[0] = run;
+}
+
+// Output for one chunk of queries: grid = (nchunks, BH).
+__global__ void __launch_bounds__(kThreads)
+    k_output(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
+             const float* __restrict__ omega, const float* __restrict__ cmax,
+             const float* __restrict__ S, float* __restrict__ out, int H, int L, int d, int M,
+             int F, int kind, int causal) {
+  extern __shared__ float sm[];
+  const int dv = d + 1;
+  float* sq = sm;                           // [kChunk][d]
+  float* sk = sq + kChunk * d;              // [kChunk][d]
+  float* sv = sk + kChunk * d;              // [kChunk][d]
+  float* sw = sv + kChunk * d;              // [kChunk]
+  float* pq = sw + kChunk;                  // [kChunk][kFeatTile]
+  float* pk = pq + kChunk * kFeatTile;      // [kChunk][kFeatTile]
+  float* sS = pk + kChunk * kFeatTile;      // [kFeatTile][dv]
+  float* A = sS + kFeatTile * dv;           // [kChunk][kChunk]
+  const int c = blockIdx.x, bh = blockIdx.y, h = bh % H;
+  const int i0 = c * kChunk, ni = min(kChunk, L - i0);
+  const size_t base = ((size_t)bh * L + i0) * d;
+  const float* om = omega + (size_t)h * M * d;
+  const float* Sc = S + (((size_t)bh * gridDim.x + (causal ? c : 0)) * F) * dv;
+  for (int i = threadIdx.x; i < kChunk * d; i += blockDim.x) {
+    const bool ok = i < ni * d;
+    sq[i] = ok ? q[base + i] : 0.f;
+    sk[i] = (ok && causal) ? k[base + i] : 0.f;
+    sv[i] = (ok && causal) ? v[base + i] : 0.f;
+  }
+  for (int i = threadIdx.x; i < kChunk * kChunk; i += blockDim.x) A[i] = 0.f;
+  __syncthreads();
+  if (causal && threadIdx.x < kChunk) {
+    const int j = threadIdx.x;
+    float w = 0.f;
+    if (j < ni) {
+      if (kind == 0) {
+        float s = 0.f;
+        for (int t = 0; t < d; ++t) s = fmaf(sk[j * d + t], sk[j * d + t], s);
+        w = expf(0.5f * s - cmax[bh]);
+      } else {
+        w = 1.f;
+      }
+    }
+    sw[j] = w;
+  }
+  // Thread mapping for the numerator: token i = tid / 4, columns n = tid % 4 + 4 m.
+  const int ti = threadIdx.x >> 2, tn = threadIdx.x & 3;
+  constexpr int kMaxCols = (kMaxD + 1 + 3) / 4;
+  float acc[kMaxCols];
+#pragma unroll
+  for (int m = 0; m < kMaxCols; ++m) acc[m] = 0.f;
+  const int nft = (F + kFeatTile - 1) / kFeatTile;
+  for (int ft = 0; ft < nft; ++ft) {
+    __syncthreads();
+    for (int p = threadIdx.x; p < kChunk * kFeatTile; p += blockDim.x) {
+      const int j = p / kFeatTile, fl = p % kFeatTile, f = ft * kFeatTile + fl;
+      float a = 0.f, b = 0.f;
+      if (j < ni && f < F) {
+        a = feature_value(kind, M, f, sq + j * d, om, d, 1.f);
+        if (causal) b = feature_value(kind, M, f, sk + j * d, om, d, sw[j]);
+      }
+      pq[p] = a;
+      pk[p] = b;
+    }
+    for (int p = threadIdx.x; p < kFeatTile * dv; p += blockDim.x) {
+      const int fl = p / dv, f = ft * kFeatTile + fl;
+      sS[p] = (f < F) ? Sc[(size_t)f * dv + (p % dv)] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < kMaxCols; ++m) {
+      const int n = tn + 4 * m;
+      if (n < dv) {
+        float s = acc[m];
+        for (int fl = 0; fl < kFeatTile; ++fl) s = fmaf(pq[ti * kFeatTile + fl], sS[fl * dv + n], s);
+        acc[m] = s;
+      }
+    }
+    if (causal) {
+      for (int p = threadIdx.x; p < kChunk * kChunk; p += blockDim.x) {
+        const int i = p / kChunk, j = p % kChunk;
+        if (j <= i) {
+          float s = A[p];
+          for (int fl = 0; fl < kFeatTile; ++fl) s = fmaf(pq[i * kFeatTile + fl], pk[j * kFeatTile + fl], s);
+          A[p] = s;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (causal) {
+#pragma unroll
+    for (int m = 0; m < kMaxCols; ++m) {
+      const int n = tn + 4 * m;
+      if (n < dv) {
+        float s = acc[m];
+        for (int j = 0; j <= ti; ++j) s = fmaf(A[ti * kChunk + j], n < d ? sv[j * d + n] : 1.f, s);
+        acc[m] = s;
+      }
+    }
+  }
+  // den lives in column d, held by thread tn == d % 4 at m = d / 4.
+  __shared__ float sden[kChunk];
+  if (tn == (d & 3)) sden[ti] = acc[d >> 2];
+  __syncthreads();
+  if (ti < ni) {
+    const float den = sden[ti];
+    const float inv = den != 0.f ? 1.f / den : 0.f;
+#pragma unroll
+    for (int m = 0; m < kMaxCols; ++m) {
+      const int n = tn + 4 * m;
+      if (n < d) out[base + (size_t)ti * d + n] = den != 0.f ? acc[m] * inv : 0.f;
+    }
+  }
+}
+
+}  // namespace f32
+
+// ------------------------------------------------------------------ ORF builder
+// One block per (head, d x d Gaussian block). Rows are orthonormalised in order by classical
+// Gram-Schmidt applied twice (fp64), then row r is scaled by |gauss_norms[h, r, :]|.
+// "Masked Language Modeling for Proteins via Linearly Scalable Long-Context Transformers"
+// (方法详解) calls these orthogonal random features. The explainer's 核心机制 section
+// constrains the directions to a random subsample of an orthogonal matrix.
+__global__ void __launch_bounds__(256)
+    k_orf(const double* __restrict__ G, const double* __restrict__ R, void* __restrict__ omega,
+          int H, int M, int d, int out_bf16) {
+  extern __shared__ double sq[];  // [d][d] rows being orthonormalised
+  __shared__ double dots[128];
+  __shared__ double snorm;
+  const int h = blockIdx.y, blk = blockIdx.x, nb = gridDim.x;
+  const double* g = G + (((size_t)h * nb + blk) * d) * d;
+  for (int i = threadIdx.x; i < d * d; i += blockDim.x) sq[i] = g[i];
+  __syncthreads();
+  for (int i = 0; i < d; ++i) {
+    double* vi = sq + (size_t)i * d;
+    for (int pass = 0; pass < 2; ++pass) {
+      if (i == 0) break;
+      // dots_j = q_j . v for j < i
+      for (int j = threadIdx.x; j < i; j += blockDim.x) {
+        const double* qj = sq + (size_t)j * d;
+        double s = 0.0;
+        for (int t = 0; t < d; ++t) s = fma(qj[t], vi[t], s);
+        dots[j] = s;
+      }
+      __syncthreads();
+      // v -= sum_j dots_j q_j
+      for (int t = threadIdx.x; t < d; t += blockDim.x) {
+        double s = 0.0;
+        for (int j = 0; j < i; ++j) s = fma(dots[j], sq[(size_t)j * d + t], s);
+        vi[t] -= s;
+      }
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+      double s = 0.0;
+      for (int t = 0; t < d; ++t) s = fma(vi[t], vi[t], s);
+      snorm = sqrt(s);
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < d; t += blockDim.x) vi[t] /= snorm;
+    __syncthreads();
+  }
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    const int r = blk * d + i;
+    if (r >= M) continue;
+    const double* rr = R + ((size_t)h * M + r) * d;
+    double s = 0.0;
+    for (int t = 0; t < d; ++t) s = fma(rr[t], rr[t], s);
+    dots[i] = sqrt(s);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < d * d; e += blockDim.x) {
+    const int i = e / d, t = e % d, r = blk * d + i;
+    if (r >= M) continue;
+    const double val = sq[e] * dots[i];
+    const size_t o = ((size_t)h * M + r) * d + t;
+    if (out_bf16)
+      reinterpret_cast<__nv_bfloat16*>(omega)[o] = __double2bfloat16(val);
+    else
+      reinterpret_cast<float*>(omega)[o] = (float)val;
+  }
+}
+
+}  // namespace favor

@@ -221,6 +221,84 @@ def row_diagnostics_head(q, k, v, Om, kind, causal, rows=None):
     return kappa, s
 
 
+def row_condition_head(q, k, v, Om, kind, causal, rows=None):
+    """Relative condition number of each chosen output row under rounding of the features.
+
+    The method computes out_i = sum_f phi_f(q_i) S_f / sum_f phi_f(q_i) z_f with
+    S_f = sum_j phi_f(k_j) v_j ([EXPL, 核心机制]). If every product phi_f(q_i) phi_f(k_j)
+    carries a relative error of at most u, then to first order
+        |d out_i| <= u (N_i + |out_i| D_i) / |den_i|,
+    with N_i = sum_f sum_j |phi_f(q_i)| |phi_f(k_j)| |v_j| and
+    D_i = sum_f sum_j |phi_f(q_i) phi_f(k_j)|. This returns
+        cond_i = (max|N_i| + max|out_i| D_i) / (|den_i| max|out_i|).
+    The trig map cancels across features as well as keys, so cond_i can reach 1e5 where
+    kappa_i is small. Causal sums run over j <= i.
+    """
+    L = q.shape[0]
+    rows = np.arange(L) if rows is None else np.asarray(rows)
+    fq = phi(q[rows], Om, kind)
+    fk = phi(k, Om, kind)
+    aq, ak, av = np.abs(fq), np.abs(fk), np.abs(v)
+    if not causal:
+        num = fq @ (fk.T @ v)
+        den = fq @ fk.sum(axis=0)
+        N = aq @ (ak.T @ av)
+        D = aq @ ak.sum(axis=0)
+    else:
+        F, dv = fk.shape[1], v.shape[1]
+        num = np.zeros((len(rows), dv))
+        den = np.zeros(len(rows))
+        N = np.zeros((len(rows), dv))
+        D = np.zeros(len(rows))
+        S, z = np.zeros((F, dv)), np.zeros(F)
+        SA, zA = np.zeros((F, dv)), np.zeros(F)
+        order = np.argsort(rows, kind="stable")
+        pos = 0
+        for j in range(L):
+            S += np.outer(fk[j], v[j])
+            z += fk[j]
+            SA += np.outer(ak[j], av[j])
+            zA += ak[j]
+            while pos < len(order) and rows[order[pos]] == j:
+                r = order[pos]
+                num[r], den[r] = fq[r] @ S, fq[r] @ z
+                N[r], D[r] = aq[r] @ SA, aq[r] @ zA
+                pos += 1
+            if pos == len(order):
+                break
+    out = _normalise(num, den)
+    on = np.abs(out).max(axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        return (np.abs(N).max(axis=1) + on * D) / (np.abs(den) * on)
+
+
+def favor_rows_head(q, k, v, Om, kind, causal, rows):
+    """FAVOR output rows `rows` of one head, by the linear-time form (prefix loop if causal)."""
+    rows = np.asarray(rows)
+    if not causal:
+        fq = phi(q[rows], Om, kind)
+        fk = phi(k, Om, kind)
+        return _normalise(fq @ (fk.T @ v), fq @ fk.sum(axis=0))
+    fq = phi(q[rows], Om, kind)
+    fk = phi(k, Om, kind)
+    S, z = np.zeros((fk.shape[1], v.shape[1])), np.zeros(fk.shape[1])
+    out = np.zeros((len(rows), v.shape[1]))
+    order = np.argsort(rows, kind="stable")
+    pos = 0
+    for j in range(q.shape[0]):
+        S += np.outer(fk[j], v[j])
+        z += fk[j]
+        while pos < len(order) and rows[order[pos]] == j:
+            r = order[pos]
+            den = fq[r] @ z
+            if den != 0.0:
+                out[r] = (fq[r] @ S) / den
+            pos += 1
+        if pos == len(order):
+            break
+    return out
+
+
 # ---------------------------------------------------------------- [B, H, L, d] wrappers
 def _per_head(fn, Q, K, V, Om, *args, **kw):
     B, H = Q.shape[:2]
@@ -260,3 +338,9 @@ def row_diagnostics(Q, K, V, Om, kind, causal, rows=None):
             s.append(c)
     L_rows = kap[0].shape[0]
     return np.stack(kap).reshape(B, H, L_rows), np.stack(s).reshape(B, H, L_rows)
+
+
+def row_condition(Q, K, V, Om, kind, causal, rows=None):
+    B, H = Q.shape[:2]
+    return np.stack([np.stack([row_condition_head(Q[b, h], K[b, h], V[b, h], Om[h], kind, causal, rows)
+                               for h in range(H)]) for b in range(B)])

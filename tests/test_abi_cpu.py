@@ -1,0 +1,76 @@
+"""The C ABI without a GPU: the library loads, exports every function include/favor.h declares,
+and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_kernelized_attention_b200 as F
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(favor_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 9, names
+    lib = ctypes.CDLL(F.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_every_declared_symbol():
+    for n in _declared():
+        assert hasattr(F, n), n
+
+
+def test_status_strings():
+    for code in range(-8, 1):
+        s = F.favor_status_string(code)
+        assert s and "unknown" not in s
+    assert "unknown" in F.favor_status_string(-99)
+
+
+def _call(**over):
+    a = dict(q=16, k=32, v=48, om=64, out=80, B=1, H=1, L=8, d=64, M=64, kind=0, causal=0)
+    a.update(over)
+    vp = ctypes.c_void_p
+    return F.lib().favor_attention(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["om"]), vp(a["out"]),
+                                   a["B"], a["H"], a["L"], a["d"], a["M"], a["kind"], a["causal"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    ({"q": 0}, -1), ({"out": 0}, -1),
+    ({"k": 33}, -2), ({"om": 8}, -2),
+    ({"L": 0}, -3), ({"B": -1}, -3), ({"M": 0}, -3), ({"d": 0}, -3),
+    ({"kind": 2}, -4), ({"kind": -1}, -4),
+])
+def test_host_validation_rejects_before_any_cuda_call(over, code):
+    # fake, never-dereferenced pointers: validation fails first, so nothing touches a device
+    assert _call(**over) == code
+
+
+def test_f32_and_orf_validation():
+    vp = ctypes.c_void_p
+    L = F.lib()
+    assert L.favor_attention_f32(None, vp(16), vp(16), vp(16), vp(16), 1, 1, 1, 1, 1, 0, 0, None) == -1
+    assert L.favor_attention_f32(vp(16), vp(16), vp(16), vp(16), vp(16), 1, 1, 1, 1, 1, 5, 0, None) == -4
+    assert L.favor_orf_omega(None, vp(16), vp(16), 1, 1, 1, 0, None) == -1
+    assert L.favor_orf_omega(vp(16), vp(24), vp(16), 1, 1, 1, 0, None) == -2
+    assert L.favor_orf_omega(vp(16), vp(16), vp(16), 0, 1, 1, 0, None) == -3
+    assert L.favor_attention_chunked(vp(16), vp(16), vp(16), vp(16), vp(16), 1, 1, 8, 64, 64, 0, 1, 7, None) in (-5, -8, -6)
+
+
+def test_workspace_bytes_is_host_only():
+    assert F.favor_workspace_bytes(1, 1, 1, 64, 64, 0, False) >= 0
+    assert F.favor_workspace_bytes(0, 1, 1, 64, 64, 0, False) == 0

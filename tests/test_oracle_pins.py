@@ -279,3 +279,33 @@ def test_error_shrinks_with_feature_count(kind):
     assert all(err[i + 1] < err[i] for i in range(len(err) - 1))
     slope = np.polyfit(np.log(Ms), np.log(err), 1)[0]
     assert -0.7 < slope < -0.35
+
+
+# ------------------------------------------------------------------ condition number used by the parity metric
+@pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
+@pytest.mark.parametrize("causal", [False, True])
+def test_row_condition_bounds_feature_perturbations(kind, causal):
+    # perturb every feature of q and k by a relative +-u: each product moves by at most ~2u, so
+    # each row may move by at most ~2u cond_i max|o_i|
+    q, k, v = _qkv(80, 16, seed=51)
+    om = _orf(32, 16, seed=51)[0]
+    rows = np.arange(80)
+    cond = O.row_condition_head(q, k, v, om, kind, causal, rows)
+    fq, fk = O.phi(q, om, kind), O.phi(k, om, kind)
+    base = O.favor_explicit_head(q, k, v, om, kind, causal)
+    u = 1e-6
+    rng = np.random.default_rng(3)
+    worst = 0.0
+    for _ in range(5):
+        pq = fq * (1 + u * rng.choice([-1.0, 1.0], fq.shape))
+        pk = fk * (1 + u * rng.choice([-1.0, 1.0], fk.shape))
+        A = pq @ pk.T
+        if causal:
+            A = np.tril(A)
+        out = (A @ v) / A.sum(axis=1, keepdims=True)
+        ratio = np.abs(out - base).max(axis=1) / (np.abs(base).max(axis=1) * 2 * u * cond)
+        worst = max(worst, ratio.max())
+    assert worst <= 1.01
+    if kind == O.RELU:
+        # all terms non-negative: D_i = den_i, so cond_i = N_i/(den_i |o_i|) + 1 is modest
+        assert cond.max() < 1e3
