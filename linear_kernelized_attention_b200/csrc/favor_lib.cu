@@ -137,27 +137,19 @@ int scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
 
 // ------------------------------------------------------------------ bf16 bidirectional plan
 struct BidirPlan {
-  int P, Mpad, nsb, Fpad, natoms, ntiles;
-  size_t part_bytes, meta_bytes, image_bytes;
+  int P, Mpad, ntiles;
 };
 
-BidirPlan plan_bidir(int BH, int L, int M, int kind) {
+// One cluster of P CTAs per head, P a power of two (<= 8, <= tiles) chosen so that B*H*P fills
+// the SMs once. The key-phase state is reduced through distributed shared memory, so the
+// bidirectional path needs no global scratch.
+BidirPlan plan_bidir(int BH, int L, int M) {
   BidirPlan pl{};
   pl.Mpad = (M + 127) / 128 * 128;
-  pl.nsb = kind == FAVOR_TRIG ? 2 * pl.Mpad / 128 : pl.Mpad / 128;
-  pl.Fpad = pl.nsb * 128;
-  pl.natoms = pl.Fpad / 64;
   pl.ntiles = (L + tc::kTile - 1) / tc::kTile;
-  int P = sm_count() / BH;
-  if (P < 1) P = 1;
-  if (P > 8) P = 8;
-  if (P > pl.ntiles) P = pl.ntiles;
+  int P = 1;
+  while (P < 8 && BH * P * 2 <= sm_count() && P * 2 <= pl.ntiles) P *= 2;
   pl.P = P;
-  if (P > 1) {
-    pl.part_bytes = (size_t)BH * P * tc::kNV * pl.Fpad * sizeof(float);
-    pl.meta_bytes = ((size_t)BH * P * 2 * sizeof(float) + 255) / 256 * 256;
-    pl.image_bytes = (size_t)BH * pl.natoms * tc::kImgAtomB;
-  }
   return pl;
 }
 
@@ -173,16 +165,12 @@ int launch_bidir_bf16(const void* q, const void* k, const void* v, const void* o
                       int B, int H, int L, int M, int kind, cudaStream_t st) {
   const int BH = B * H;
   if (BH > 65535 * 8) return FAVOR_ERR_UNSUPPORTED;
-  const BidirPlan pl = plan_bidir(BH, L, M, kind);
+  const BidirPlan pl = plan_bidir(BH, L, M);
   CUtensorMap mq, mk, mv, mo, mom;
   if (!make_map_rows64(&mq, q, L, BH) || !make_map_rows64(&mk, k, L, BH) ||
       !make_map_rows64(&mv, v, L, BH) || !make_map_rows64(&mo, out, L, BH) ||
       !make_map_rows64(&mom, omega, M, H))
     return FAVOR_ERR_CUDA;
-  void* ws = nullptr;
-  const size_t ws_bytes = pl.part_bytes + pl.meta_bytes + pl.image_bytes;
-  int rc = scratch_alloc(&ws, ws_bytes, st);
-  if (rc != FAVOR_OK) return rc;
   tc::BidirParams prm{};
   prm.BH = BH;
   prm.H = H;
@@ -191,31 +179,26 @@ int launch_bidir_bf16(const void* q, const void* k, const void* v, const void* o
   prm.Mpad = pl.Mpad;
   prm.P = pl.P;
   prm.ntiles = pl.ntiles;
-  uint8_t* w = static_cast<uint8_t*>(ws);
-  prm.part = reinterpret_cast<float*>(w);
-  prm.pmeta = reinterpret_cast<float*>(w + pl.part_bytes);
-  prm.image = w + pl.part_bytes + pl.meta_bytes;
   const uint32_t smem = tc::bidir_smem_bytes(pl.Mpad);
-  auto kern = kind == FAVOR_TRIG ? tc::favor_bidir_tc<0> : tc::favor_bidir_tc<1>;
+  // Trig keys use 32-token slices; ReLU uses 64-token slices when its state (<= 2 blocks of
+  // 128 features) leaves TMEM room for them.
+  auto kern = kind == FAVOR_TRIG ? tc::favor_bidir_tc<0, 32>
+              : (pl.Mpad <= 256 ? tc::favor_bidir_tc<1, 64> : tc::favor_bidir_tc<1, 32>);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    rc = FAVOR_ERR_CUDA;
-  if (rc == FAVOR_OK) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(BH * pl.P, 1, 1);
-    cfg.blockDim = dim3(tc::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = pl.P;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mom, mo, prm) != cudaSuccess) rc = FAVOR_ERR_CUDA;
-  }
-  if (ws) cudaFreeAsync(ws, st);
-  return rc;
+    return FAVOR_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(BH * pl.P, 1, 1);
+  cfg.blockDim = dim3(tc::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = pl.P;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mom, mo, prm) == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ fp32 path
@@ -289,10 +272,10 @@ int favor_sync_status(void* stream) {
 
 size_t favor_workspace_bytes(int B, int H, int L, int d, int M, int feature_kind, int causal) {
   if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || M <= 0) return 0;
-  (void)d;
+  (void)feature_kind;
   (void)causal;
-  const BidirPlan pl = plan_bidir(B * H, L, M, feature_kind);
-  return pl.part_bytes + pl.meta_bytes + pl.image_bytes;
+  (void)d;
+  return 0;  // the bidirectional tensor-core path reduces through distributed shared memory
 }
 
 int favor_attention_chunked(const void* q, const void* k, const void* v, const void* omega,

@@ -90,8 +90,12 @@ def test_bidir_constant_v_and_zero_queries():
     c.v = fi.as_f64(c.t[2])
     c._dev = None
     for kind in (0, 1):
-        g = _run(c, kind)
-        np.testing.assert_allclose(g, np.broadcast_to(fi.as_f64(val), g.shape), rtol=2e-2, atol=2e-2)
+        g = _run(c, kind).reshape(2, 500, 64)
+        ref, cond, _ = c.oracle(kind, False)
+        # the exact answer is the constant row; trig rows with heavy cancellation get the
+        # condition-aware allowance like every other parity check
+        np.testing.assert_allclose(ref, np.broadcast_to(fi.as_f64(val), ref.shape), rtol=1e-9, atol=1e-9)
+        check_rows(g, ref, cond, TOL_BF16, U_BF16, f"constant v kind={kind}")
     # ReLU with q = 0: every feature of q is 0, so the denominator is 0 and the row is 0
     c.t[0] = torch.zeros_like(c.t[0])
     c._dev = None
