@@ -163,118 +163,48 @@ __device__ __forceinline__ void load_state_cols(uint32_t taddr, float (&v)[40]) 
   for (int e = 0; e < 8; ++e) v[32 + e] = __uint_as_float(b[e]);
 }
 
-// KIND: 0 trig, 1 ReLU. IW: key-phase slice width in tokens (32 or 64).
+// Everything the key phase needs from its kernel.
+struct KeyCtx {
+  uint8_t* gbase;                 // generic pointer to the 1024-aligned shared base
+  uint32_t base, s_om, s_reg;     // shared-space addresses
+  uint32_t tmem;                  // TMEM base (512 columns)
+  int tid, warp, lane;
+  int h, bh, t_begin, my_tiles, L, Mpad;
+  int nblk, nsb, ipt, kUK, kPK;
+};
+
+// Key phase (see the file comment): accumulates the CTA's partial state in TMEM columns
+// [0, nsb * 80) and commits ms->s_done when the last state MMA completes. Trig also leaves the
+// final stabiliser reference in ms->cfinal. Every warp of the CTA calls this.
 template <int KIND, int IW>
-__global__ void __launch_bounds__(kThreads, 1)
-    favor_bidir_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_om,
-                   const __grid_constant__ CUtensorMap tm_out, const BidirParams p) {
-  static_assert(IW == 32 || IW == 64, "key slice width");
-  static_assert(KIND == 1 || IW == 32, "trig uses 32-token key slices");
-  constexpr int NH = IW / 32;                       // 32-column sub-items per key item
-  constexpr int PW = KIND == 0 ? IW : IW / 2;       // key phi slot width (packed 16-bit)
-  constexpr int PWQ = KIND == 0 ? 64 : 32;          // query phi slot width
-  constexpr int SPT = kTile / IW;                   // key slices per tile
-
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t s_om = base;
-  const uint32_t s_reg = base + uint32_t(p.Mpad) * kRowB;
-  Misc* ms = reinterpret_cast<Misc*>(gbase + (s_reg + kRegionB - base));
+__device__ __forceinline__ void key_phase(const KeyCtx& kc, Misc* ms, const CUtensorMap* tm_k,
+                                          const CUtensorMap* tm_v, const CUtensorMap* tm_q,
+                                          const CUtensorMap* tm_om) {
+  constexpr int NH = IW / 32;
+  constexpr int PW = KIND == 0 ? IW : IW / 2;
+  constexpr int SPT = kTile / IW;
+  uint8_t* const gbase = kc.gbase;
+  const uint32_t base = kc.base, s_om = kc.s_om, s_reg = kc.s_reg, tmem = kc.tmem;
+  const int warp = kc.warp, lane = kc.lane;
+  const int h = kc.h, bh = kc.bh, t_begin = kc.t_begin, my_tiles = kc.my_tiles;
+  const int nblk = kc.nblk, nsb = kc.nsb, ipt = kc.ipt, kUK = kc.kUK, kPK = kc.kPK;
   volatile int* abort_flag = &ms->abort_flag;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int P = p.P;
-  const int rank = blockIdx.x % P;
-  const int bh = blockIdx.x / P;
-  const int h = bh % p.H;
-  const int t_begin = rank * p.ntiles / P;
-  const int my_tiles = (rank + 1) * p.ntiles / P - t_begin;
-  const int nblk = p.Mpad / 128;               // key-phase angle blocks
-  const int nsb = KIND == 0 ? 2 * nblk : nblk; // state blocks of 128 feature rows
-  const int Fpad = nsb * 128;
-  const int natoms = Fpad / 64;
-  const int ipt = nblk * SPT;                  // key-phase items per tile
-  const int nchq = p.Mpad / 64;                // query-phase chunks per tile (even)
-  const int kUK = nsb * kNPad;                 // key-phase U ring base, then the phi ring
-  const int kPK = kUK + kNU * IW;
   auto bar = [](uint64_t& b) { return smem_u32(&b); };
-
-  // ---------------------------------------------------------------- set-up
-  if (tid == 0) {
-    ms->abort_flag = 0;
-    mbar_init(bar(ms->om_full), 1);
-    for (int s = 0; s < kStagesK; ++s) {
-      mbar_init(bar(ms->kv_full[s]), 1);
-      mbar_init(bar(ms->kv_empty[s]), KIND == 0 ? 2 : 1);
-      mbar_init(bar(ms->w_full[s]), 32);
-    }
-    for (int b = 0; b < kNU; ++b) {
-      mbar_init(bar(ms->u_full[b]), 1);
-      mbar_init(bar(ms->u_free[b]), 4);
-      mbar_init(bar(ms->uq_full[b]), 1);
-      mbar_init(bar(ms->uq_free[b]), 4);
-    }
-    for (int b = 0; b < kNPK; ++b) {
-      mbar_init(bar(ms->p_full[b]), 4);
-      mbar_init(bar(ms->p_free[b]), 1);
-    }
-    for (int b = 0; b < kNPQ; ++b) {
-      mbar_init(bar(ms->pq_full[b]), 4);
-      mbar_init(bar(ms->pq_free[b]), 1);
-    }
-    mbar_init(bar(ms->s_done), 1);
-    mbar_init(bar(ms->img_full), 1);
-    mbar_init(bar(ms->mma_drain), 1);
-    mbar_init(bar(ms->mma_drain1), 1);
-    for (int s = 0; s < kStagesQ; ++s) {
-      mbar_init(bar(ms->q_full[s]), 1);
-      mbar_init(bar(ms->q_empty[s]), 1);
-    }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(ms->num_full[s]), 1);
-      mbar_init(bar(ms->num_empty[s]), 4);
-      mbar_init(bar(ms->out_sync[s]), 128);
-    }
-    mbar_init(bar(ms->epi_sync), 256);
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(&ms->tmem_base), 512);
-    tmem_relinquish();
-  }
-  {  // column buffers for [V | w]: zero, and for ReLU a constant 1.0 in column 64 of every row
-    uint4* col = reinterpret_cast<uint4*>(gbase + (s_reg + kColOff - base));
-    const int n16 = (KIND == 0 ? kStagesK : 1) * kTileB / 16;
-    for (int i = tid; i < n16; i += kThreads) col[i] = make_uint4(0u, 0u, 0u, 0u);
-    __syncthreads();
-    if (KIND == 1 && tid < kTile)
-      reinterpret_cast<uint16_t*>(gbase + (s_reg + kColOff - base) + tid * kRowB + ((tid & 7) << 4))[0] = 0x3F80u;
-    fence_proxy_async_smem();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = ms->tmem_base;
-
-  // ================================================================ key phase
   if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_q);
-      mbar_arrive_expect_tx(bar(ms->om_full), uint32_t(p.Mpad) * kRowB);
+      tma_prefetch_desc(tm_k);
+      tma_prefetch_desc(tm_v);
+      tma_prefetch_desc(tm_q);
+      mbar_arrive_expect_tx(bar(ms->om_full), uint32_t(kc.Mpad) * kRowB);
       for (int blk = 0; blk < nblk; ++blk)
-        tma_load_3d(s_om + blk * kTileB, &tm_om, bar(ms->om_full), 0, blk * 128, h);
+        tma_load_3d(s_om + blk * kTileB, tm_om, bar(ms->om_full), 0, blk * 128, h);
       for (int t = 0; t < my_tiles; ++t) {
         const int s = t % kStagesK, k = t / kStagesK;
         if (!mbar_wait(bar(ms->kv_empty[s]), (k & 1) ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar(ms->kv_full[s]), 2 * kTileB);
         const int row = (t_begin + t) * kTile;
-        tma_load_3d(s_reg + s * 2 * kTileB, &tm_k, bar(ms->kv_full[s]), 0, row, bh);
-        tma_load_3d(s_reg + s * 2 * kTileB + kTileB, &tm_v, bar(ms->kv_full[s]), 0, row, bh);
+        tma_load_3d(s_reg + s * 2 * kTileB, tm_k, bar(ms->kv_full[s]), 0, row, bh);
+        tma_load_3d(s_reg + s * 2 * kTileB + kTileB, tm_v, bar(ms->kv_full[s]), 0, row, bh);
       }
     }
     __syncwarp();
@@ -386,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               acc = fmaf(hi, hi, acc);
             }
           }
-          n2[jj] = row0 + j < p.L ? 0.5f * acc : -INFINITY;
+          n2[jj] = row0 + j < kc.L ? 0.5f * acc : -INFINITY;
           m = fmaxf(m, n2[jj]);
         }
 #pragma unroll
@@ -506,6 +436,129 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(have = step(ua, ub))) break;
       have = step(ub, ua);
     }
+  }
+
+}
+
+// KIND: 0 trig, 1 ReLU. IW: key-phase slice width in tokens (32 or 64).
+template <int KIND, int IW>
+__global__ void __launch_bounds__(kThreads, 1)
+    favor_bidir_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_om,
+                   const __grid_constant__ CUtensorMap tm_out, const BidirParams p) {
+  static_assert(IW == 32 || IW == 64, "key slice width");
+  static_assert(KIND == 1 || IW == 32, "trig uses 32-token key slices");
+  constexpr int NH = IW / 32;                       // 32-column sub-items per key item
+  constexpr int PW = KIND == 0 ? IW : IW / 2;       // key phi slot width (packed 16-bit)
+  constexpr int PWQ = KIND == 0 ? 64 : 32;          // query phi slot width
+  constexpr int SPT = kTile / IW;                   // key slices per tile
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t s_om = base;
+  const uint32_t s_reg = base + uint32_t(p.Mpad) * kRowB;
+  Misc* ms = reinterpret_cast<Misc*>(gbase + (s_reg + kRegionB - base));
+  volatile int* abort_flag = &ms->abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int P = p.P;
+  const int rank = blockIdx.x % P;
+  const int bh = blockIdx.x / P;
+  const int h = bh % p.H;
+  const int t_begin = rank * p.ntiles / P;
+  const int my_tiles = (rank + 1) * p.ntiles / P - t_begin;
+  const int nblk = p.Mpad / 128;               // key-phase angle blocks
+  const int nsb = KIND == 0 ? 2 * nblk : nblk; // state blocks of 128 feature rows
+  const int Fpad = nsb * 128;
+  const int natoms = Fpad / 64;
+  const int ipt = nblk * SPT;                  // key-phase items per tile
+  const int nchq = p.Mpad / 64;                // query-phase chunks per tile (even)
+  const int kUK = nsb * kNPad;                 // key-phase U ring base, then the phi ring
+  const int kPK = kUK + kNU * IW;
+  auto bar = [](uint64_t& b) { return smem_u32(&b); };
+
+  // ---------------------------------------------------------------- set-up
+  if (tid == 0) {
+    ms->abort_flag = 0;
+    mbar_init(bar(ms->om_full), 1);
+    for (int s = 0; s < kStagesK; ++s) {
+      mbar_init(bar(ms->kv_full[s]), 1);
+      mbar_init(bar(ms->kv_empty[s]), KIND == 0 ? 2 : 1);
+      mbar_init(bar(ms->w_full[s]), 32);
+    }
+    for (int b = 0; b < kNU; ++b) {
+      mbar_init(bar(ms->u_full[b]), 1);
+      mbar_init(bar(ms->u_free[b]), 4);
+      mbar_init(bar(ms->uq_full[b]), 1);
+      mbar_init(bar(ms->uq_free[b]), 4);
+    }
+    for (int b = 0; b < kNPK; ++b) {
+      mbar_init(bar(ms->p_full[b]), 4);
+      mbar_init(bar(ms->p_free[b]), 1);
+    }
+    for (int b = 0; b < kNPQ; ++b) {
+      mbar_init(bar(ms->pq_full[b]), 4);
+      mbar_init(bar(ms->pq_free[b]), 1);
+    }
+    mbar_init(bar(ms->s_done), 1);
+    mbar_init(bar(ms->img_full), 1);
+    mbar_init(bar(ms->mma_drain), 1);
+    mbar_init(bar(ms->mma_drain1), 1);
+    for (int s = 0; s < kStagesQ; ++s) {
+      mbar_init(bar(ms->q_full[s]), 1);
+      mbar_init(bar(ms->q_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(ms->num_full[s]), 1);
+      mbar_init(bar(ms->num_empty[s]), 4);
+      mbar_init(bar(ms->out_sync[s]), 128);
+    }
+    mbar_init(bar(ms->epi_sync), 256);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ms->tmem_base), 512);
+    tmem_relinquish();
+  }
+  {  // column buffers for [V | w]: zero, and for ReLU a constant 1.0 in column 64 of every row
+    uint4* col = reinterpret_cast<uint4*>(gbase + (s_reg + kColOff - base));
+    const int n16 = (KIND == 0 ? kStagesK : 1) * kTileB / 16;
+    for (int i = tid; i < n16; i += kThreads) col[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    if (KIND == 1 && tid < kTile)
+      reinterpret_cast<uint16_t*>(gbase + (s_reg + kColOff - base) + tid * kRowB + ((tid & 7) << 4))[0] = 0x3F80u;
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+
+  // ================================================================ key phase
+  {
+    KeyCtx kc;
+    kc.gbase = gbase;
+    kc.base = base;
+    kc.s_om = s_om;
+    kc.s_reg = s_reg;
+    kc.tmem = tmem;
+    kc.tid = tid;
+    kc.warp = warp;
+    kc.lane = lane;
+    kc.h = h;
+    kc.bh = bh;
+    kc.t_begin = t_begin;
+    kc.my_tiles = my_tiles;
+    kc.L = p.L;
+    kc.Mpad = p.Mpad;
+    kc.nblk = nblk;
+    kc.nsb = nsb;
+    kc.ipt = ipt;
+    kc.kUK = kUK;
+    kc.kPK = kPK;
+    key_phase<KIND, IW>(kc, ms, &tm_k, &tm_v, &tm_q, &tm_om);
   }
 
   // ================================================================ state reduction
