@@ -14,6 +14,7 @@
 #include "ptx.cuh"
 #include "kernels_f32.cuh"
 #include "kernel_bidir.cuh"
+#include "kernel_causal.cuh"
 
 namespace favor {
 
@@ -201,6 +202,52 @@ int launch_bidir_bf16(const void* q, const void* k, const void* v, const void* o
   return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mom, mo, prm) == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ bf16 causal
+// Feature blocks per head: 64 angles (trig) or 128 angles (ReLU) per CTA; 3 rounds up to 4 so
+// that the cluster's row ownership (rows of warp quarter q go to CTA q % G) is balanced.
+int causal_blocks(int M, int kind) {
+  int G = kind == FAVOR_TRIG ? (M + 63) / 64 : (M + 127) / 128;
+  return G == 3 ? 4 : G;
+}
+
+int launch_causal_bf16(const void* q, const void* k, const void* v, const void* omega, void* out,
+                       int B, int H, int L, int M, int kind, cudaStream_t st) {
+  const int BH = B * H;
+  const int G = causal_blocks(M, kind);
+  if (G < 1 || G > 4) return FAVOR_ERR_UNSUPPORTED;
+  if ((long long)BH * G > INT_MAX) return FAVOR_ERR_UNSUPPORTED;
+  CUtensorMap mq, mk, mv, mom;
+  if (!make_map_rows64(&mq, q, L, BH) || !make_map_rows64(&mk, k, L, BH) ||
+      !make_map_rows64(&mv, v, L, BH) || !make_map_rows64(&mom, omega, M, H))
+    return FAVOR_ERR_CUDA;
+  tc::CausalParams prm{};
+  prm.BH = BH;
+  prm.H = H;
+  prm.L = L;
+  prm.M = M;
+  prm.G = G;
+  prm.nch = (L + tc::kTile - 1) / tc::kTile;
+  const uint32_t smem = tc::causal_smem_bytes();
+  auto kern = kind == FAVOR_TRIG ? tc::favor_causal_tc<0> : tc::favor_causal_tc<1>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return FAVOR_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(BH * G, 1, 1);
+  cfg.blockDim = dim3(tc::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = G;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mom, prm, static_cast<__nv_bfloat16*>(out)) == cudaSuccess
+             ? FAVOR_OK
+             : FAVOR_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ fp32 path
 size_t f32_workspace(int BH, int L, int d, int M, int kind) {
   const int F = kind == FAVOR_TRIG ? 2 * M : M;
@@ -285,9 +332,11 @@ int favor_attention_chunked(const void* q, const void* k, const void* v, const v
   if (rc != FAVOR_OK) return rc;
   if ((rc = check_device()) != FAVOR_OK) return rc;
   if ((rc = check_tc_shape(d, M, feature_kind)) != FAVOR_OK) return rc;
-  if (chunk != 0 && chunk != 64 && chunk != 128) return FAVOR_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (causal) return FAVOR_ERR_UNSUPPORTED;
+  if (causal) {
+    if (chunk != 0 && chunk != tc::kTile) return FAVOR_ERR_UNSUPPORTED;
+    return launch_causal_bf16(q, k, v, omega, out, B, H, L, M, feature_kind, st);
+  }
   return launch_bidir_bf16(q, k, v, omega, out, B, H, L, M, feature_kind, st);
 }
 

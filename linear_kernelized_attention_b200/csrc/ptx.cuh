@@ -79,6 +79,39 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// Cluster-scope acquire variant of the bounded wait, for barriers that other CTAs of the
+// cluster arrive on (their shared-memory writes before the arrive become visible).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (abort && *abort) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      record_error(-7 /* FAVOR_ERR_TIMEOUT */);
+      if (abort) *abort = 1;
+      return false;
+    }
+  }
+}
+// Arrive on an mbarrier of another CTA of the cluster (address from mapa_shared). Release at
+// cluster scope: this thread's earlier writes, shared::cluster stores included, are visible to
+// a thread that observes the phase with an acquire.cluster wait.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+
 // Bounded barrier among the `count` threads an mbarrier was initialised with: arrive, then
 // wait for the phase to complete. `phase` is this thread's running phase bit.
 __device__ __forceinline__ bool group_sync(uint32_t bar, uint32_t& phase, volatile int* abort) {
@@ -135,6 +168,11 @@ __device__ __forceinline__ float2 ld_dsmem_f2(uint32_t addr) {
   float2 v;
   asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
   return v;
+}
+__device__ __forceinline__ void st_dsmem_f4(uint32_t addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
 }
 __device__ __forceinline__ void st_dsmem_u2(uint32_t addr, uint32_t a, uint32_t b) {
   asm volatile("st.shared::cluster.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
@@ -303,6 +341,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[30]), "r"(r[31])
       : "memory");
 }
+
+// ------------------------------------------------------------------ arithmetic
+// 2^x by the SFU's approximate base-2 exponential (PTX ex2.approx.ftz.f32); 2^x = 0 for very
+// negative x.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// 2^e for an integer e in [-126, 127], exactly.
+__device__ __forceinline__ float pow2i(int e) { return __uint_as_float(uint32_t(127 + e) << 23); }
 
 // ------------------------------------------------------------------ packing
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
