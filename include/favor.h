@@ -127,6 +127,30 @@ int favor_attention_host(const void* q, const void* k, const void* v, const void
                          void* out, int B, int H, int L, int d, int M, int feature_kind,
                          int causal, int dtype_code, void* stream);
 
+/*
+ * fp32 forward pass that allocates nothing (no counterpart on the pages: an interface for
+ * callers that cannot allocate device memory). Same arguments, arithmetic and results as
+ * favor_attention_f32, whose kernels it launches, but the workspace lives in a static
+ * device array of favor_noalloc_scratch_bytes() bytes (32 MiB) that belongs to the library,
+ * one per device. No cudaMalloc, cudaMallocAsync, cudaFree or allocating library routine is
+ * called.
+ *   Size limit: the workspace is B*H*ceil(L/64)*F*(d+1)*4 + B*H*4 bytes (F = 2M for trig,
+ *   M for ReLU). A call whose workspace exceeds the array returns FAVOR_ERR_UNSUPPORTED and
+ *   launches nothing.
+ *   Overlap: every call on a device uses the same array. Calls whose executions overlap (on
+ *   different streams, or from different host threads without ordering between their streams)
+ *   race on it and give undefined results. Order them on one stream or with events.
+ *   First call: it looks up the array's device address with cudaGetSymbolAddress, once per
+ *   device, and returns FAVOR_ERR_CUDA if that fails. Make a first call on each device before
+ *   any stream capture begins.
+ */
+int favor_attention_f32_noalloc(const float* q, const float* k, const float* v, const float* omega,
+                                float* out, int B, int H, int L, int d, int M, int feature_kind,
+                                int causal, void* stream);
+
+/* Size in bytes of the static workspace of favor_attention_f32_noalloc. */
+size_t favor_noalloc_scratch_bytes(void);
+
 /* Synchronise `stream`, then read and clear the device status word (FAVOR_OK or a code). */
 int favor_sync_status(void* stream);
 

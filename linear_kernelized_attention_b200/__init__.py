@@ -7,7 +7,7 @@ if the library is missing or a call fails, an exception is raised.
 Entry points mirror the C ABI in include/favor.h:
     favor_attention, favor_attention_chunked, favor_attention_f32, favor_orf_omega,
     favor_attention_host, favor_sync_status, favor_status_string, favor_workspace_bytes,
-    favor_selftest_timeout
+    favor_selftest_timeout, favor_attention_f32_noalloc, favor_noalloc_scratch_bytes
 """
 from __future__ import annotations
 
@@ -34,6 +34,8 @@ _SIGS = {
     "favor_status_string": (ctypes.c_char_p, [_i]),
     "favor_selftest_timeout": (_i, [_ll, _vp]),
     "favor_workspace_bytes": (_sz, [_i] * 7),
+    "favor_attention_f32_noalloc": (_i, [_vp] * 5 + [_i] * 7 + [_vp]),
+    "favor_noalloc_scratch_bytes": (_sz, []),
 }
 _LIB = None
 
@@ -172,3 +174,23 @@ def favor_workspace_bytes(B, H, L, d, M, feature_kind=FAVOR_TRIG, causal=False) 
 
 def favor_selftest_timeout(limit_cycles: int, stream=None) -> int:
     return lib().favor_selftest_timeout(int(limit_cycles), _stream(stream))
+
+
+def favor_attention_f32_noalloc(q, k, v, omega, out=None, feature_kind=FAVOR_TRIG, causal=False,
+                                stream=None):
+    """fp32 forward with its workspace in the library's static device array (no allocation by
+    the library; `out` is allocated here only if not given). Calls that overlap in time race on
+    the shared workspace: see include/favor.h."""
+    import torch
+    B, H, L, d, M = _check_qkv(q, k, v, omega, torch.float32)
+    if out is None:
+        out = torch.empty_like(q)
+    rc = lib().favor_attention_f32_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), omega.data_ptr(),
+                                           out.data_ptr(), B, H, L, d, M, int(feature_kind), int(causal),
+                                           _stream(stream))
+    _check(rc, "favor_attention_f32_noalloc")
+    return out
+
+
+def favor_noalloc_scratch_bytes() -> int:
+    return lib().favor_noalloc_scratch_bytes()

@@ -290,6 +290,67 @@ int launch_f32(const float* q, const float* k, const float* v, const float* omeg
 
 }  // namespace
 
+// ------------------------------------------------------------------ allocation-free fp32 entry
+namespace favor {
+// Scratch of favor_attention_f32_noalloc: a static device array, so that entry point needs no
+// allocation. One array per device, shared by every call on that device.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+}  // namespace favor
+
+namespace {
+
+// Device address of the static scratch on the current device, looked up once per device.
+int noalloc_scratch(void** p) {
+  static void* addr[64] = {};
+  static std::mutex mu;
+  *p = nullptr;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FAVOR_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return FAVOR_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(mu);
+  if (!addr[dev]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, favor::g_noalloc_scratch) != cudaSuccess || !a) return FAVOR_ERR_CUDA;
+    addr[dev] = a;
+  }
+  *p = addr[dev];
+  return FAVOR_OK;
+}
+
+// The fp32 path's launch sequence with its workspace in the static scratch.
+int launch_f32_static(const float* q, const float* k, const float* v, const float* omega, float* out,
+                      int B, int H, int L, int d, int M, int kind, int causal, cudaStream_t st) {
+  const int BH = B * H;
+  const int F = kind == FAVOR_TRIG ? 2 * M : M;
+  const int nch = (L + f32::kChunk - 1) / f32::kChunk;
+  const int nft = (F + f32::kFeatTile - 1) / f32::kFeatTile;
+  if (BH > 65535 || nch > 65535) return FAVOR_ERR_UNSUPPORTED;
+  if (f32_workspace(BH, L, d, M, kind) > favor::kNoAllocScratchBytes) return FAVOR_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  int rc = noalloc_scratch(&ws);
+  if (rc != FAVOR_OK) return rc;
+  float* dS = static_cast<float*>(ws);
+  float* cmax = dS + (size_t)BH * nch * F * (d + 1);
+  const size_t sm_state = (size_t)(2 * f32::kChunk * d + f32::kChunk + f32::kChunk * f32::kFeatTile) * 4;
+  const size_t sm_out = (size_t)(3 * f32::kChunk * d + f32::kChunk + 2 * f32::kChunk * f32::kFeatTile +
+                                 f32::kFeatTile * (d + 1) + f32::kChunk * f32::kChunk) * 4;
+  if (cudaFuncSetAttribute(f32::k_chunk_state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_state) != cudaSuccess ||
+      cudaFuncSetAttribute(f32::k_output, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out) != cudaSuccess)
+    return FAVOR_ERR_CUDA;
+  if (kind == FAVOR_TRIG) f32::k_key_halfnorm_max<<<BH, f32::kThreads, 0, st>>>(k, cmax, L, d);
+  f32::k_chunk_state<<<dim3(nft, nch, BH), f32::kThreads, sm_state, st>>>(k, v, omega, cmax, dS, H, L, d, M, F,
+                                                                           kind);
+  const long long per_chunk = (long long)F * (d + 1);
+  const long long total = (long long)BH * per_chunk;
+  f32::k_scan_chunks<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(dS, nch, per_chunk, total, causal);
+  f32::k_output<<<dim3(nch, BH), f32::kThreads, sm_out, st>>>(q, k, v, omega, cmax, dS, out, H, L, d, M, F, kind,
+                                                              causal);
+  return cudaGetLastError() == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
+}
+
+}  // namespace
+
 // ====================================================================== C ABI
 extern "C" {
 
@@ -412,6 +473,19 @@ int favor_attention_host(const void* q, const void* k, const void* v, const void
   if (cudaStreamSynchronize(st) != cudaSuccess && rc == FAVOR_OK) rc = FAVOR_ERR_CUDA;
   return rc;
 }
+
+int favor_attention_f32_noalloc(const float* q, const float* k, const float* v, const float* omega,
+                                float* out, int B, int H, int L, int d, int M, int feature_kind,
+                                int causal, void* stream) {
+  int rc = check_common(q, k, v, omega, out, B, H, L, d, M, feature_kind);
+  if (rc != FAVOR_OK) return rc;
+  if ((rc = check_device()) != FAVOR_OK) return rc;
+  if (d > f32::kMaxD || M > 512) return FAVOR_ERR_UNSUPPORTED;
+  return launch_f32_static(q, k, v, omega, out, B, H, L, d, M, feature_kind, causal,
+                           static_cast<cudaStream_t>(stream));
+}
+
+size_t favor_noalloc_scratch_bytes(void) { return favor::kNoAllocScratchBytes; }
 
 // Launch the bounded-wait self-test: a wait that nothing satisfies, limited to `limit_cycles`.
 // favor_sync_status() afterwards must report FAVOR_ERR_TIMEOUT.
