@@ -28,7 +28,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 WORKLOAD = dict(B=4, H=8, L=4096, d=64, M=256)
-VARIANTS = [("trig_bidir", 0, False), ("relu_bidir", 1, False)]
+VARIANTS = [("trig_bidir", 0, False), ("relu_bidir", 1, False), ("trig_causal", 0, True), ("relu_causal", 1, True)]
 N_SETS = 4
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "FAVOR fwd tokens/s (B·H·L/s) at L=4096,d=64,M=256; % of tensor/HBM roofline"

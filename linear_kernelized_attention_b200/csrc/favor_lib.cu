@@ -53,10 +53,34 @@ int check_device() {
 }
 
 int sm_count() {
+  static int cache[64] = {};
   int dev = 0, n = 148;
   cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (dev >= 0 && dev < 64) cache[dev] = n;
   return n;
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device): the attribute
+// persists, and setting it on every call costs host time on the launch path.
+int ensure_smem_attr(const void* kern, int bytes) {
+  struct Entry {
+    const void* k;
+    int dev, bytes;
+  };
+  static Entry done[64];
+  static int n = 0;
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FAVOR_ERR_CUDA;
+  std::lock_guard<std::mutex> g(mu);
+  for (int i = 0; i < n; ++i)
+    if (done[i].k == kern && done[i].dev == dev && done[i].bytes >= bytes) return FAVOR_OK;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return FAVOR_ERR_CUDA;
+  if (n < 64) done[n++] = Entry{kern, dev, bytes};
+  return FAVOR_OK;
 }
 
 // Common shape/pointer checks shared by every entry point.
@@ -185,8 +209,7 @@ int launch_bidir_bf16(const void* q, const void* k, const void* v, const void* o
   // 128 features) leaves TMEM room for them.
   auto kern = kind == FAVOR_TRIG ? tc::favor_bidir_tc<0, 32>
               : (pl.Mpad <= 256 ? tc::favor_bidir_tc<1, 64> : tc::favor_bidir_tc<1, 32>);
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return FAVOR_ERR_CUDA;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)smem) != FAVOR_OK) return FAVOR_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(BH * pl.P, 1, 1);
   cfg.blockDim = dim3(tc::kThreads, 1, 1);
@@ -229,8 +252,7 @@ int launch_causal_bf16(const void* q, const void* k, const void* v, const void* 
   prm.nch = (L + tc::kTile - 1) / tc::kTile;
   const uint32_t smem = tc::causal_smem_bytes();
   auto kern = kind == FAVOR_TRIG ? tc::favor_causal_tc<0> : tc::favor_causal_tc<1>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return FAVOR_ERR_CUDA;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)smem) != FAVOR_OK) return FAVOR_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(BH * G, 1, 1);
   cfg.blockDim = dim3(tc::kThreads, 1, 1);
