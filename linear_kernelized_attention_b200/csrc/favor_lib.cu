@@ -226,10 +226,14 @@ int launch_bidir_bf16(const void* q, const void* k, const void* v, const void* o
 }
 
 // ------------------------------------------------------------------ bf16 causal
-// Feature blocks per head: 64 angles (trig) or 128 angles (ReLU) per CTA; 3 rounds up to 4 so
-// that the cluster's row ownership (rows of warp quarter q go to CTA q % G) is balanced.
+// Angles per CTA: 64 (trig; ReLU with M <= 256) or 128 (ReLU with M > 256).
+int causal_angles(int M, int kind) { return kind == FAVOR_RELU && M > 256 ? 128 : 64; }
+
+// CTAs per head; 3 rounds up to 4 so that the cluster's row ownership (rows of warp quarter q go
+// to CTA q % G) is balanced.
 int causal_blocks(int M, int kind) {
-  int G = kind == FAVOR_TRIG ? (M + 63) / 64 : (M + 127) / 128;
+  const int na = causal_angles(M, kind);
+  const int G = (M + na - 1) / na;
   return G == 3 ? 4 : G;
 }
 
@@ -251,11 +255,12 @@ int launch_causal_bf16(const void* q, const void* k, const void* v, const void* 
   prm.G = G;
   prm.nch = (L + tc::kTile - 1) / tc::kTile;
   const uint32_t smem = tc::causal_smem_bytes();
-  auto kern = kind == FAVOR_TRIG ? tc::favor_causal_tc<0> : tc::favor_causal_tc<1>;
+  auto kern = kind == FAVOR_TRIG ? tc::favor_causal_tc<0, 64>
+              : (causal_angles(M, kind) == 64 ? tc::favor_causal_tc<1, 64> : tc::favor_causal_tc<1, 128>);
   if (ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)smem) != FAVOR_OK) return FAVOR_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(BH * G, 1, 1);
-  cfg.blockDim = dim3(tc::kThreads, 1, 1);
+  cfg.blockDim = dim3(tc::kThreadsC, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];

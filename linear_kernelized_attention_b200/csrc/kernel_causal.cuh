@@ -9,102 +9,116 @@
 //   S_{<c+1} = S_{<c} + phi(K_c)^T [V_c | 1].
 // The first term ("inter") reads the state; the second ("intra") is a masked 128 x 128 product.
 //
-// Parallel split. One thread-block cluster of G CTAs per (batch, head); CTA g owns a block of
-// 128 features (trig: 64 angles as interleaved cos/sin pairs; ReLU: 128 angles), so every CTA
-// walks the whole sequence with a 128 x 80 state slab in TMEM. num and den are sums over
-// features, so the G partial rows add; CTA (q4 % G) owns rows 32 q4 .. 32 q4 + 31 of a chunk
-// and receives the other CTAs' partials through distributed shared memory.
+// Parallel split. One thread-block cluster of G CTAs per (batch, head); CTA g owns one block of
+// NA angles (trig: 64 angles as 128 interleaved cos/sin features; ReLU: NA = 64 or 128 angles,
+// one feature each, padded with zero features to 128), so every CTA walks the whole sequence with
+// a 128-feature state slab in TMEM. num and den are sums over features, so the G partial rows
+// add: every CTA deposits its partial rows of a chunk (numerators in bf16, the denominator in
+// fp32; two deposit buffers by chunk parity) with the CTA that owns them (rows 32 q .. 32 q + 31
+// belong to CTA q % G), and a combiner warp there sums, divides and stores.
 //
 // Stabiliser (trig). Key features carry exp(|k_j|^2/2). The state S_{<c} is kept relative to
 // the running reference cref_c = max |k_j|^2/2 over earlier chunks; row i of chunk c uses its
 // own reference R_i = max(cref_c, max_{j <= i in c} |k_j|^2/2), so every weight is <= 1 and no
 // row's terms vanish under another row's larger keys:
 //   intra_ij = P_ij exp(|k_j|^2/2 - R_i), inter_i scaled by exp(cref_c - R_i).
-// After chunk c the state is rescaled to cnew_c = max(cref_c, chunk max) before the chunk's keys
-// (weighted exp(|k_j|^2/2 - cnew_c)) are added. Factors that cancel in the ratio (1/sqrt(M),
-// exp(|q|^2/2)) are dropped. ReLU uses unit weights.
+// The key weight is folded into the stored key features, phi'(k_j) = a_j phi(k_j):
+//   usual chunks: a_j = exp(|k_j|^2/2 - cnew_c), cnew_c = max(cref_c, chunk max). Then
+//     P' = phi(Q) phi'(K)^T needs only the causal mask, the row factor rho_i = exp(cnew_c - R_i)
+//     is applied to the intra sums once, and S += phi'(K)^T [V | 1] reads the V tile as it is.
+//   chunks whose keys rise more than 2^80 above R_0 (e.g. the first large key of a sequence):
+//     a_j = exp(|k_j|^2/2 - R_j), P16_ij = P'_ij exp(R_j - R_i) per element, and the state update
+//     uses [u o V | u] with u_j = exp(R_j - cnew_c). A weight that underflows there is below 2^-46
+//     of its row's largest weight.
+// After chunk c the state is rescaled from cref_c to cnew_c before the chunk's keys are added.
+// Factors that cancel in the ratio (1/sqrt(M), exp(|q|^2/2)) are dropped. ReLU uses unit weights.
 //
-// Per chunk (MMAs issued by one thread; fp32 accumulation in TMEM):
-//   U_K = K_c Omega_g^T      bf16, M=128 keys, N=64 angles per slice  -> phi(K) fp16 in smem
-//   U_Q = Q_c Omega_g^T      bf16, M=128 queries, N=64/128           -> phi(Q) fp16 in TMEM
-//   P = phi(Q) phi(K)^T      fp16, N=128 keys
-//   inter = phi(Q) S_img     fp16 image of S_{<c} (power-of-two scale), N=64
-//   S += phi(K)^T [w o V | w]  fp16, M=128 features, N=80
-//   intra = P16 V_c          P16 = weighted, masked P in bf16 (TMEM), V_c the bf16 tile, N=64
-// Denominators are accumulated in fp32 registers: phi(q_i).z (z = the state's normaliser
-// column, kept in fp32) and sum_j P16_ij.
+// Per chunk (bf16 operands, fp32 accumulation in TMEM):
+//   issuer A:  U_K = K_c Omega_g^T (N=64 per slice)            -> phi'(K) in smem (2 buffers)
+//              S += phi'(K)^T V  (M=128 features, N=64)        z += phi'(K)^T 1  (N=16)
+//   issuer B:  U_Q = Q_c Omega_g^T (N=NA)                      -> phi(Q) in TMEM (in place)
+//              P' = phi(Q) phi'(K)^T (N=128), inter = phi(Q) S_img (bf16 image of S_{<c}),
+//              intra = P16 V_c (P16 = masked P' in TMEM; V_c the TMA tile)
+//              phi(Q).z with z (the normaliser column of S_{<c}) split into bf16 hi and lo parts,
+//              rows 0 and 1 of a 16-row operand
+// The intra denominator sum_j P16_ij is accumulated in fp32 registers.
 //
-// Warp roles (384 threads): 0 TMA; 1 TMEM allocator and MMA issuer; 3 key norms, references
-// and [w o V | w]; 4-7 key features and the state image (thread = key / feature row);
-// 8-11 query features, P16, output and the cluster exchange (thread = query row).
+// Warp roles (416 threads): 0 TMA; 1 TMEM allocator and issuer A; 2 issuer B; 3 key norms and
+// references; 4-7 state image and phi'(K) (thread = feature / key row); 8-11 phi(Q), P16 and
+// partial rows (thread = query row); 12 combiner of the owned rows.
 #pragma once
 #include "kernel_bidir.cuh"
 
 namespace favor {
 namespace tc {
 
+constexpr int kThreadsC = 416;
 // Shared memory (offsets from the 1024-aligned base).
 constexpr int kC_OM = 0;              // Omega rows of this CTA's angles (one 128-row box)
-constexpr int kC_K = 16 * 1024;       // K stages, 2 x 16 KB
-constexpr int kC_V = 48 * 1024;       // V stages, 2 x 16 KB (V_c stays until its intra MMA)
-constexpr int kC_Q = 80 * 1024;       // Q stage
-constexpr int kC_PHK = 96 * 1024;     // phi(K) fp16: 2 atoms of 64 features x 128 keys
-constexpr int kC_VW = 128 * 1024;     // [w o V] fp16, the V tile's layout
-constexpr int kC_COL = 144 * 1024;    // column buffer: w (trig) or 1 (ReLU) as column 64
-constexpr int kC_IMG = 160 * 1024;    // state image fp16: 128 feature rows x 64 values
-constexpr int kC_RECV = 176 * 1024;   // partial rows received from the cluster (<= 26 KB)
-constexpr int kC_SMALL = 202 * 1024;  // per-chunk scalars and vectors (CausalSmall)
-constexpr int kC_MISC = 206 * 1024;   // barriers (CausalMisc)
-constexpr int kRecvRowB = 68 * 4;     // one partial row: 64 numerators, the denominator, pad
+constexpr int kC_K = 16 * 1024;       // K tile
+constexpr int kC_V = 32 * 1024;       // V stages, 2 x 16 KB (V_c stays until its intra MMA)
+constexpr int kC_Q = 64 * 1024;       // Q tile
+constexpr int kC_PHK = 80 * 1024;     // phi(K): 2 buffers x 2 atoms of 64 features x 128 keys
+constexpr int kPhkB = 2 * kTileB;     // one phi(K) buffer
+constexpr int kC_VW = 144 * 1024;     // [u o V] bf16 (trig, large-rise chunks), the V tile's layout
+constexpr int kC_WROW = 160 * 1024;   // 1 (or u) as row 0 of a 16 x 128 K-major operand (2 x 2 KB)
+constexpr int kC_ZROW = 164 * 1024;   // z of S_{<c} (hi, lo) as rows 0, 1 of a 16 x 128 operand
+constexpr int kC_IMG = 168 * 1024;    // state image bf16: 128 feature rows x 64 values
+constexpr int kC_RECV = 184 * 1024;   // partial rows deposited for the rows this CTA owns
+constexpr int kRecvRowB = 144;        // one partial row: 64 bf16 numerators, fp32 denominator, pad
+constexpr int kRecvBufB = 4 * 32 * kRecvRowB;  // 128 row slots (owned quarters x senders x 32)
+constexpr int kRecvB = 2 * kRecvBufB;          // two buffers, by chunk parity
+constexpr int kC_SMALL = kC_RECV + kRecvB;  // per-chunk scalars and vectors (CausalSmall)
+constexpr int kC_MISC = kC_SMALL + 5120;    // barriers (CausalMisc)
+constexpr int kMeta = 4;                     // chunks of key metadata in flight
 // TMEM columns.
-constexpr uint32_t kT_S = 0;          // state slab, 80 columns (lanes = features)
+constexpr uint32_t kT_S = 0;          // state slab: 64 value columns + 16 (column 64 = z)
 constexpr uint32_t kT_PR = 80;        // P (128 fp32) -> P16 [80, 144) + intra [144, 208)
-constexpr uint32_t kT_IN = 208;       // inter accumulator, 64 columns
-constexpr uint32_t kT_A = 272;        // U_Q (64 / 128 columns) -> phi(Q) packed fp16 (64)
-constexpr uint32_t kT_B = 400;        // U_K slice, 64 columns
+constexpr uint32_t kT_IN = 208;       // inter accumulator (64 columns) + phi(Q).z (16; column 64)
+constexpr uint32_t kT_A = 288;        // U_Q (NA columns) -> phi(Q) packed bf16 (64)
+constexpr uint32_t kT_B = 416;        // U_K slice, 64 columns
 
 struct CausalParams {
   int BH, H, L, M;   // heads (B*H), heads per batch, tokens, random features
-  int G;             // CTAs per head (feature blocks): 1, 2 or 4
+  int G;             // CTAs per head (angle blocks): 1, 2 or 4
   int nch;           // ceil(L / 128)
 };
 
 struct CausalSmall {
-  float z[128];           // normaliser column of S_{<c}, fp32
-  float n2l[2][128];      // |k_j|^2/2 * log2(e) of the chunk's keys, by chunk parity
-  float rl[2][128];       // row references R_i * log2(e), by chunk parity
-  float crefl[2], cnewl[2];  // references of S_{<c} and S_{<=c} (log2 units)
-  float imgexp[2];        // image scale exponent of S_{<c}
-  float red[2][4];        // per-warp max |S| for the image scale
+  float rl[kMeta][128];      // row references R_i * log2(e), by chunk % kMeta
+  float wk[kMeta][128];      // key feature weights a_j, by chunk % kMeta
+  float crefl[kMeta], cnewl[kMeta];  // references of S_{<c} and S_{<=c} (log2 units)
+  int fb[kMeta];             // 1: the chunk takes the large-rise weights
 };
-static_assert(sizeof(CausalSmall) <= 4096, "causal small block");
-static_assert(kC_RECV + 3 * 32 * kRecvRowB <= kC_SMALL, "receive buffer");
+static_assert(sizeof(CausalSmall) <= 5120, "causal small block");
 
 struct alignas(16) CausalMisc {
   int abort_flag;
   uint32_t tmem_base;
   int pad[2];
-  uint64_t om_full, kv_full[2], kv_empty[2], q_full, q_empty;
-  uint64_t meta_full[2], meta_free[2], vw_full;
-  uint64_t uk_full, uk_free, uq_full, p_full, inter_done, s_done, o_full, drain;
-  uint64_t img_full, img_free, s_ready, phik_full, phiq_full, p16_full, pr_free;
-  uint64_t ksync;
-  uint64_t recv_full[4], recv_free[4];
+  uint64_t om_full, k_full, k_empty, v_full[2], v_empty[2], q_full, q_empty;
+  uint64_t meta_full[kMeta], meta_free[kMeta], vw_full;
+  uint64_t uk_full, uk_free, uq_full, p_full, inter_done, s_done, o_full, drain_a, drain_b;
+  uint64_t img_full, img_free, s_ready, phiq_full, p16_full, pr_free;
+  uint64_t phik_full[2], phik_free[2];  // per phi(K) buffer
+  uint64_t recv_full[4][2], recv_free[4][2];  // per row quarter and deposit buffer
 };
 static_assert(sizeof(CausalMisc) <= 1024, "causal misc block");
 
 __host__ __device__ constexpr uint32_t causal_smem_bytes() { return kC_MISC + 1024 + 1024; }
 
-// KIND: 0 trig, 1 ReLU.
-template <int KIND>
-__global__ void __launch_bounds__(kThreads, 1)
+// KIND: 0 trig, 1 ReLU. NA: angles per CTA (trig 64; ReLU 64 or 128).
+template <int KIND, int NA>
+__global__ void __launch_bounds__(kThreadsC, 1)
     favor_causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_om,
                     const CausalParams p, __nv_bfloat16* __restrict__ out) {
-  constexpr int NA = KIND == 0 ? 64 : 128;  // angles per CTA
-  constexpr int NSL = NA / 64;              // 64-angle slices of the key projection
+  static_assert(NA == 64 || (KIND == 1 && NA == 128), "angles per CTA");
+  constexpr int NSL = NA / 64;                  // 64-angle slices of the key projection
+  constexpr bool kHalfFeat = KIND == 1 && NA == 64;  // features 64..127 of the block are zero
   constexpr float kLog2e = 1.4426950408889634f;
-  constexpr float kNegBig = -1.0e30f;       // reference before any key; weight of padded keys
+  constexpr float kNegBig = -1.0e30f;           // reference before any key; weight of padded keys
+  constexpr float kSplitMax = 80.f;             // largest reference jump (log2) for w_j rho_i
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -125,11 +139,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     ms->abort_flag = 0;
     mbar_init(bar(ms->om_full), 1);
+    mbar_init(bar(ms->k_full), 1);
+    mbar_init(bar(ms->k_empty), 2);        // key-norm warp + issuer A (U_K)
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(ms->kv_full[s]), 1);
-      mbar_init(bar(ms->kv_empty[s]), 2);  // key-norm warp + the intra MMA's commit
-      mbar_init(bar(ms->meta_full[s]), 32);
-      mbar_init(bar(ms->meta_free[s]), 4);
+      mbar_init(bar(ms->v_full[s]), 1);
+      mbar_init(bar(ms->v_empty[s]), 3);   // key-norm warp + issuer A (S) + issuer B (intra)
+    }
+    for (int b = 0; b < kMeta; ++b) {
+      mbar_init(bar(ms->meta_full[b]), 32);
+      mbar_init(bar(ms->meta_free[b]), 4);
     }
     mbar_init(bar(ms->q_full), 1);
     mbar_init(bar(ms->q_empty), 1);
@@ -141,31 +159,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(ms->inter_done), 1);
     mbar_init(bar(ms->s_done), 1);
     mbar_init(bar(ms->o_full), 1);
-    mbar_init(bar(ms->drain), 1);
+    mbar_init(bar(ms->drain_a), 1);
+    mbar_init(bar(ms->drain_b), 1);
     mbar_init(bar(ms->img_full), 4);
-    mbar_init(bar(ms->img_free), 1 + 4);  // inter MMA commit + the 4 query warps (z read)
+    mbar_init(bar(ms->img_free), 1);      // issuer B's commit after the inter and z MMAs
     mbar_init(bar(ms->s_ready), 4);
-    mbar_init(bar(ms->phik_full), 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(ms->phik_full[b]), 4);
+      mbar_init(bar(ms->phik_free[b]), 1);  // issuer B's commit after P
+    }
     mbar_init(bar(ms->phiq_full), 4);
     mbar_init(bar(ms->p16_full), 4);
     mbar_init(bar(ms->pr_free), 4);
-    mbar_init(bar(ms->ksync), 128);
-    for (int q = 0; q < 4; ++q) {
-      mbar_init(bar(ms->recv_full[q]), G > 1 ? 32 * (G - 1) : 1);
-      mbar_init(bar(ms->recv_free[q]), 32);
-    }
+    for (int q = 0; q < 4; ++q)
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(bar(ms->recv_full[q][b]), 32 * G);  // 32 lanes of every CTA of the cluster
+        mbar_init(bar(ms->recv_free[q][b]), 32);      // the owner's combiner lanes
+      }
     fence_mbar_init();
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&ms->tmem_base), 512);
     tmem_relinquish();
   }
-  {  // column buffer: zero; ReLU: fp16 1.0 in column 64 of every key row
-    uint4* col = reinterpret_cast<uint4*>(gb + kC_COL);
-    for (int i = tid; i < kTileB / 16; i += kThreads) col[i] = make_uint4(0u, 0u, 0u, 0u);
+  {  // phi(K) buffers zero (the padded features of a half-filled block stay zero); the w row
+     // operand zero except row 0, which is 1 (trig large-rise chunks rewrite it)
+    uint4* phk = reinterpret_cast<uint4*>(gb + kC_PHK);
+    for (int i = tid; i < 2 * kPhkB / 16; i += kThreadsC) phk[i] = make_uint4(0u, 0u, 0u, 0u);
+    uint4* wr = reinterpret_cast<uint4*>(gb + kC_WROW);  // the w and z operands, 8 KB
+    for (int i = tid; i < 8192 / 16; i += kThreadsC) wr[i] = make_uint4(0u, 0u, 0u, 0u);
     __syncthreads();
-    if (KIND == 1 && tid < kTile)
-      reinterpret_cast<uint16_t*>(gb + kC_COL + tid * kRowB + ((tid & 7) << 4))[0] = 0x3C00u;
+    if (tid < kTile) *reinterpret_cast<uint16_t*>(gb + kC_WROW + (tid >> 6) * 2048 + (tid & 63) * 2) = 0x3F80u;
     fence_proxy_async_smem();
   }
   tc_fence_before();
@@ -173,6 +197,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (G > 1) cluster_sync();  // the partners' barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
+
+  const uint32_t id_uk = idesc_f16(128, 64, 1, 1, 0, 0);
+  const uint32_t id_uq = idesc_f16(128, NA, 1, 1, 0, 0);
+  const uint32_t id_p = idesc_f16(128, 128, 1, 1, 0, 0);
+  const uint32_t id_in = idesc_f16(128, 64, 1, 1, 0, 1);
+  const uint32_t id_s = idesc_f16(128, 64, 1, 1, 1, 1);
+  const uint32_t id_z = idesc_f16(128, 16, 1, 1, 1, 0);
+  const uint32_t id_qz = idesc_f16(128, 16, 1, 1, 0, 0);
+  const uint32_t id_it = idesc_f16(128, 64, 1, 1, 0, 1);
+  constexpr uint64_t kKStep = (16 * kRowB) >> 4;  // 16 rows of an MN-major operand
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -182,14 +216,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_q);
       mbar_arrive_expect_tx(bar(ms->om_full), kTileB);
       tma_load_3d(base + kC_OM, &tm_om, bar(ms->om_full), 0, g * NA, h);
-      int kv_issued = 0, q_issued = 0;
+      int k_issued = 0, v_issued = 0, q_issued = 0;
       for (int c = 0; c < nch; ++c) {
         const int s = c & 1;
-        if (c >= 2 && !mbar_wait(bar(ms->kv_empty[s]), ((c >> 1) - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(ms->kv_full[s]), 2 * kTileB);
-        tma_load_3d(base + kC_K + s * kTileB, &tm_k, bar(ms->kv_full[s]), 0, c * kTile, bh);
-        tma_load_3d(base + kC_V + s * kTileB, &tm_v, bar(ms->kv_full[s]), 0, c * kTile, bh);
-        kv_issued = c + 1;
+        if (c >= 1 && !mbar_wait(bar(ms->k_empty), (c - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(ms->k_full), kTileB);
+        tma_load_3d(base + kC_K, &tm_k, bar(ms->k_full), 0, c * kTile, bh);
+        k_issued = c + 1;
+        if (c >= 2 && !mbar_wait(bar(ms->v_empty[s]), ((c >> 1) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(ms->v_full[s]), kTileB);
+        tma_load_3d(base + kC_V + s * kTileB, &tm_v, bar(ms->v_full[s]), 0, c * kTile, bh);
+        v_issued = c + 1;
         if (c >= 1 && !mbar_wait(bar(ms->q_empty), (c - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar(ms->q_full), kTileB);
         tma_load_3d(base + kC_Q, &tm_q, bar(ms->q_full), 0, c * kTile, bh);
@@ -197,121 +234,146 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // On an abort, let the copies already issued land before the CTA can exit.
       if (*abort_flag) {
-        mbar_wait(bar(ms->om_full), 0, nullptr, kWaitLimitCycles / 8);
-        for (int c = kv_issued > 2 ? kv_issued - 2 : 0; c < kv_issued; ++c)
-          mbar_wait(bar(ms->kv_full[c & 1]), (c >> 1) & 1, nullptr, kWaitLimitCycles / 8);
-        if (q_issued > 0) mbar_wait(bar(ms->q_full), (q_issued - 1) & 1, nullptr, kWaitLimitCycles / 8);
+        constexpr long long kDrain = kWaitLimitCycles / 8;
+        mbar_wait(bar(ms->om_full), 0, nullptr, kDrain);
+        if (k_issued > 0) mbar_wait(bar(ms->k_full), (k_issued - 1) & 1, nullptr, kDrain);
+        for (int c = v_issued > 2 ? v_issued - 2 : 0; c < v_issued; ++c)
+          mbar_wait(bar(ms->v_full[c & 1]), (c >> 1) & 1, nullptr, kDrain);
+        if (q_issued > 0) mbar_wait(bar(ms->q_full), (q_issued - 1) & 1, nullptr, kDrain);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ issuer A: U_K, S and z
     if (lane == 0) {
-      const uint32_t id_uk = idesc_f16(128, 64, 1, 1, 0, 0);
-      const uint32_t id_uq = idesc_f16(128, NA, 1, 1, 0, 0);
-      const uint32_t id_p = idesc_f16(128, 128, 0, 0, 0, 0);
-      const uint32_t id_in = idesc_f16(128, 64, 0, 0, 0, 1);
-      const uint32_t id_s = idesc_f16(128, kNPad, 0, 0, 1, 1);
-      const uint32_t id_it = idesc_f16(128, 64, 1, 1, 0, 1);
       const uint64_t d_om = sdesc_sw128(base + kC_OM, 16, 1024);
-      const uint64_t d_q = sdesc_sw128(base + kC_Q, 16, 1024);
-      const uint64_t d_k0 = sdesc_sw128(base + kC_K, 16, 1024);
+      const uint64_t d_k = sdesc_sw128(base + kC_K, 16, 1024);
+      const uint64_t d_phk_a = sdesc_sw128(base + kC_PHK, kTileB, 1024);  // MN-major A of S, z
+      const uint64_t d_vw = sdesc_sw128(base + kC_VW, kTileB, 1024);
       const uint64_t d_v0 = sdesc_sw128(base + kC_V, kTileB, 1024);
-      const uint64_t d_phk_b = sdesc_sw128(base + kC_PHK, 16, 1024);      // K-major B of P
-      const uint64_t d_phk_a = sdesc_sw128(base + kC_PHK, kTileB, 1024);  // MN-major A of S
-      const uint64_t d_img = sdesc_sw128(base + kC_IMG, kTileB, 1024);
-      const uint64_t d_vw = sdesc_sw128(base + kC_VW, kC_COL - kC_VW, 1024);
-      constexpr uint64_t kKStep = (16 * kRowB) >> 4;  // 16 rows of an MN-major operand
-      auto intra = [&](int cc) -> bool {
-        if (!mbar_wait(bar(ms->p16_full), cc & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint64_t bv = d_v0 + uint64_t(((cc & 1) * kTileB) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + kT_PR + 64, tmem + kT_PR + 8 * kk, bv + kk * kKStep, id_it, kk > 0 ? 1u : 0u);
-        mma_commit(bar(ms->o_full));
-        mma_commit(bar(ms->kv_empty[cc & 1]));
-        return true;
-      };
-      bool ok = mbar_wait(bar(ms->om_full), 0, abort_flag);
+      const uint64_t d_wr = sdesc_sw128(base + kC_WROW, 16, 1024);        // K-major B of z
       uint32_t ukc = 0;
-      for (int c = 0; ok && c < nch; ++c) {
-        const int s = c & 1;
-        // U_K(c), one 64-angle slice at a time
-        if (!(ok = mbar_wait(bar(ms->kv_full[s]), (c >> 1) & 1, abort_flag))) break;
+      auto uk = [&](int c) -> bool {
+        if (!mbar_wait(bar(ms->k_full), c & 1, abort_flag)) return false;
         for (int sl = 0; sl < NSL; ++sl) {
-          if (ukc > 0 && !(ok = mbar_wait(bar(ms->uk_free), (ukc - 1) & 1, abort_flag))) break;
+          if (ukc > 0 && !mbar_wait(bar(ms->uk_free), (ukc - 1) & 1, abort_flag)) return false;
           tc_fence_after();
-          const uint64_t a = d_k0 + uint64_t((s * kTileB) >> 4);
           const uint64_t b = d_om + uint64_t((sl * 64 * kRowB) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + kT_B, a + 2 * kk, b + 2 * kk, id_uk, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + kT_B, d_k + 2 * kk, b + 2 * kk, id_uk, kk > 0 ? 1u : 0u);
           mma_commit(bar(ms->uk_full));
           ++ukc;
         }
-        if (!ok) break;
-        // U_Q(c) into the phi(Q) region, once P(c-1) and inter(c-1) have read phi(Q_{c-1})
-        if (!(ok = mbar_wait(bar(ms->q_full), c & 1, abort_flag))) break;
-        if (c >= 1 && !(ok = mbar_wait(bar(ms->inter_done), (c - 1) & 1, abort_flag))) break;
+        mma_commit(bar(ms->k_empty));  // the K tile has been read
+        return true;
+      };
+      bool ok = mbar_wait(bar(ms->om_full), 0, abort_flag) && (nch == 0 || uk(0));
+      for (int c = 0; ok && c < nch; ++c) {
+        // S += phi(K)^T [w o V], z += phi(K)^T w
+        if (!(ok = mbar_wait(bar(ms->phik_full[c & 1]), (c >> 1) & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(bar(ms->s_ready), c & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(bar(ms->vw_full), c & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint64_t a = d_phk_a + uint64_t(((c & 1) * kPhkB) >> 4);
+        const bool use_vw = KIND == 0 && sm->fb[c & (kMeta - 1)];
+        const uint64_t bvw = use_vw ? d_vw : d_v0 + uint64_t(((c & 1) * kTileB) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
+          mma_ss(tmem + kT_S, a + kk * kKStep, bvw + kk * kKStep, id_s, acc);
+          mma_ss(tmem + kT_S + 64, a + kk * kKStep, d_wr + uint64_t(((kk >> 2) * 2048 + (kk & 3) * 32) >> 4), id_z,
+                 acc);
+        }
+        mma_commit(bar(ms->s_done));
+        mma_commit(bar(ms->v_empty[c & 1]));  // the V tile has been read
+        if (c + 1 < nch && !(ok = uk(c + 1))) break;
+      }
+      mma_commit(bar(ms->drain_a));
+      mbar_wait(bar(ms->drain_a), 0, nullptr, kWaitLimitCycles / 8);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ issuer B: U_Q, P, inter, intra
+    if (lane == 0) {
+      const uint64_t d_om = sdesc_sw128(base + kC_OM, 16, 1024);
+      const uint64_t d_q = sdesc_sw128(base + kC_Q, 16, 1024);
+      const uint64_t d_v0 = sdesc_sw128(base + kC_V, kTileB, 1024);
+      const uint64_t d_phk_b = sdesc_sw128(base + kC_PHK, 16, 1024);  // K-major B of P
+      const uint64_t d_img = sdesc_sw128(base + kC_IMG, kTileB, 1024);
+      const uint64_t d_zr = sdesc_sw128(base + kC_ZROW, 16, 1024);  // K-major B of phi(Q).z
+      auto uq = [&](int c) -> bool {
+        if (!mbar_wait(bar(ms->q_full), c & 1, abort_flag)) return false;
+        if (c >= 1 && !mbar_wait(bar(ms->inter_done), (c - 1) & 1, abort_flag)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + kT_A, d_q + 2 * kk, d_om + 2 * kk, id_uq, kk > 0 ? 1u : 0u);
         mma_commit(bar(ms->uq_full));
         mma_commit(bar(ms->q_empty));
-        // intra(c-1)
-        if (c >= 1 && !(ok = intra(c - 1))) break;
+        return true;
+      };
+      bool ok = mbar_wait(bar(ms->om_full), 0, abort_flag) && (nch == 0 || uq(0));
+      for (int c = 0; ok && c < nch; ++c) {
         // P(c) = phi(Q) phi(K)^T
-        if (!(ok = mbar_wait(bar(ms->phik_full), c & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(bar(ms->phik_full[c & 1]), (c >> 1) & 1, abort_flag))) break;
         if (!(ok = mbar_wait(bar(ms->phiq_full), c & 1, abort_flag))) break;
         if (c >= 1 && !(ok = mbar_wait(bar(ms->pr_free), (c - 1) & 1, abort_flag))) break;
         tc_fence_after();
+        const uint64_t bk = d_phk_b + uint64_t(((c & 1) * kPhkB) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + kT_PR, tmem + kT_A + 8 * kk, d_phk_b + uint64_t(((kk >> 2) * kTileB + (kk & 3) * 32) >> 4),
-                 id_p, kk > 0 ? 1u : 0u);
+          mma_ts(tmem + kT_PR, tmem + kT_A + 8 * kk, bk + uint64_t(((kk >> 2) * kTileB + (kk & 3) * 32) >> 4), id_p,
+                 kk > 0 ? 1u : 0u);
         mma_commit(bar(ms->p_full));
-        // inter(c) = phi(Q) S_img
+        mma_commit(bar(ms->phik_free[c & 1]));
+        // inter(c) = phi(Q) S_img and phi(Q).z
         if (!(ok = mbar_wait(bar(ms->img_full), c & 1, abort_flag))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
+        for (int kk = 0; kk < 8; ++kk) {
           mma_ts(tmem + kT_IN, tmem + kT_A + 8 * kk, d_img + kk * kKStep, id_in, kk > 0 ? 1u : 0u);
+          mma_ts(tmem + kT_IN + 64, tmem + kT_A + 8 * kk, d_zr + uint64_t(((kk >> 2) * 2048 + (kk & 3) * 32) >> 4),
+                 id_qz, kk > 0 ? 1u : 0u);
+        }
         mma_commit(bar(ms->inter_done));
         mma_commit(bar(ms->img_free));
-        // S += phi(K)^T [w o V | w]
-        if (!(ok = mbar_wait(bar(ms->s_ready), c & 1, abort_flag))) break;
-        if (!(ok = mbar_wait(bar(ms->vw_full), c & 1, abort_flag))) break;
+        // U_Q(c+1) into the phi(Q) region, once P(c) and inter(c) have read phi(Q_c)
+        if (c + 1 < nch && !(ok = uq(c + 1))) break;
+        // intra(c) = P16 V_c
+        if (!(ok = mbar_wait(bar(ms->p16_full), c & 1, abort_flag))) break;
         tc_fence_after();
+        const uint64_t bv = d_v0 + uint64_t(((c & 1) * kTileB) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + kT_S, d_phk_a + kk * kKStep, d_vw + kk * kKStep, id_s, (c > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar(ms->s_done));
+          mma_ts(tmem + kT_PR + 64, tmem + kT_PR + 8 * kk, bv + kk * kKStep, id_it, kk > 0 ? 1u : 0u);
+        mma_commit(bar(ms->o_full));
+        mma_commit(bar(ms->v_empty[c & 1]));  // the V tile has been read
       }
-      if (ok && nch > 0) intra(nch - 1);
-      // every MMA issued has completed before TMEM can be released
-      mma_commit(bar(ms->drain));
-      mbar_wait(bar(ms->drain), 0, nullptr, kWaitLimitCycles / 8);
+      mma_commit(bar(ms->drain_b));
+      mbar_wait(bar(ms->drain_b), 0, nullptr, kWaitLimitCycles / 8);
     }
     __syncwarp();
   } else if (warp == 3) {
-    // ------------------------------------------------------------ key norms, references, [w o V | w]
+    // ------------------------------------------------------------ key norms and references
     float crefl = kNegBig;
+    bool prev_fb = false;
     for (int c = 0; c < nch; ++c) {
-      const int s = c & 1, pz = c & 1;
-      if (!mbar_wait(bar(ms->kv_full[s]), (c >> 1) & 1, abort_flag)) break;
-      if (c >= 2 && !mbar_wait(bar(ms->meta_free[pz]), ((c >> 1) - 1) & 1, abort_flag)) break;
-      const uint8_t* kt = gb + kC_K + s * kTileB;
+      const int s = c & 1, mb = c & (kMeta - 1);
+      if (!mbar_wait(bar(ms->k_full), c & 1, abort_flag)) break;
+      if (c >= kMeta && !mbar_wait(bar(ms->meta_free[mb]), ((c / kMeta) - 1) & 1, abort_flag)) break;
       const int row0 = c * kTile;
-      float nl[4];
       float cnewl = 0.f;
+      bool fb = false;
       if (KIND == 0) {
-#pragma unroll
+        // |k_j|^2/2 (log2 units; kept in wk until the weights are known) and R_j, the
+        // inclusive prefix max over the chunk's keys in order, seeded with cref
+        float run = crefl;
+#pragma unroll 1
         for (int jj = 0; jj < 4; ++jj) {
           const int j = lane + 32 * jj;
           float acc = 0.f;
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
-            const uint4 x = *reinterpret_cast<const uint4*>(kt + j * kRowB + ((ch ^ (j & 7)) << 4));
+            const uint4 x = *reinterpret_cast<const uint4*>(gb + kC_K + j * kRowB + ((ch ^ (j & 7)) << 4));
             const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -320,125 +382,200 @@ __global__ void __launch_bounds__(kThreads, 1)
               acc = fmaf(hi, hi, acc);
             }
           }
-          nl[jj] = row0 + j < L ? 0.5f * acc * kLog2e : kNegBig;
-        }
-        // R_i: inclusive prefix max over the chunk's keys in order, seeded with cref
-        float run = crefl;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          float x = nl[jj];
+          const float nl = row0 + j < L ? 0.5f * acc * kLog2e : kNegBig;
+          float x = nl;
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) {
             const float y = __shfl_up_sync(0xffffffffu, x, o);
             if (lane >= o) x = fmaxf(x, y);
           }
           x = fmaxf(x, run);
-          sm->n2l[pz][lane + 32 * jj] = nl[jj];
-          sm->rl[pz][lane + 32 * jj] = x;
+          sm->rl[mb][j] = x;
+          sm->wk[mb][j] = nl;
           run = __shfl_sync(0xffffffffu, x, 31);
         }
         cnewl = run;
-      } else {
+        __syncwarp();
+        // every R_i >= R_0, so rho_i = 2^(cnewl - rl_i) <= 2^(cnewl - R_0)
+        fb = cnewl - sm->rl[mb][0] > kSplitMax;
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) nl[jj] = 0.f;
+        for (int jj = 0; jj < 4; ++jj) {
+          const int j = lane + 32 * jj;
+          sm->wk[mb][j] = ex2_approx(sm->wk[mb][j] - (fb ? sm->rl[mb][j] : cnewl));
+        }
       }
       if (lane == 0) {
-        sm->crefl[pz] = crefl;
-        sm->cnewl[pz] = cnewl;
+        sm->crefl[mb] = crefl;
+        sm->cnewl[mb] = cnewl;
+        sm->fb[mb] = fb ? 1 : 0;
       }
-      mbar_arrive(bar(ms->meta_full[pz]));
-      // [w o V] and w, once the previous state update has read the buffers
+      mbar_arrive(bar(ms->meta_full[mb]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(ms->k_empty));
+      if (!mbar_wait(bar(ms->v_full[s]), (c >> 1) & 1, abort_flag)) break;
+      // the previous state update has read [u o V] and the w row (this also keeps vw_full at
+      // most one phase ahead of its waiter)
       if (c >= 1 && !mbar_wait(bar(ms->s_done), (c - 1) & 1, abort_flag)) break;
-      const uint8_t* vt = gb + kC_V + s * kTileB;
-      uint8_t* vw = gb + kC_VW;
+      if (KIND == 0 && (fb || prev_fb)) {
+        // large-rise chunk: [u o V] and u in row 0 of the w operand; the next chunk restores 1
+        const uint8_t* vt = gb + kC_V + s * kTileB;
+#pragma unroll 1
+        for (int jj = 0; jj < 4; ++jj) {
+          const int j = lane + 32 * jj;
+          const float u = fb ? ex2_approx(sm->rl[mb][j] - cnewl) : 1.f;
+          if (fb) {
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int j = lane + 32 * jj;
-        const float w = KIND == 0 ? ex2_approx(nl[jj] - cnewl) : 1.f;  // 0 for padded keys
+            for (int ch = 0; ch < 8; ++ch) {
+              const uint32_t off = j * kRowB + ((ch ^ (j & 7)) << 4);
+              const uint4 x = *reinterpret_cast<const uint4*>(vt + off);
+              const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+              uint32_t o4[4];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint32_t off = j * kRowB + ((ch ^ (j & 7)) << 4);
-          const uint4 x = *reinterpret_cast<const uint4*>(vt + off);
-          const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
-          uint32_t o4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            o4[e] = pack_f16x2(__uint_as_float(w4[e] << 16) * w, __uint_as_float(w4[e] & 0xFFFF0000u) * w);
-          *reinterpret_cast<uint4*>(vw + off) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+              for (int e = 0; e < 4; ++e)
+                o4[e] = pack_bf16x2(__uint_as_float(w4[e] << 16) * u, __uint_as_float(w4[e] & 0xFFFF0000u) * u);
+              *reinterpret_cast<uint4*>(gb + kC_VW + off) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            }
+          }
+          *reinterpret_cast<__nv_bfloat16*>(gb + kC_WROW + (j >> 6) * 2048 + (j & 63) * 2) = __float2bfloat16_rn(u);
         }
-        if (KIND == 0)
-          *reinterpret_cast<__half*>(gb + kC_COL + j * kRowB + ((j & 7) << 4)) = __float2half_rn(w);
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
+      prev_fb = fb;
       mbar_arrive(bar(ms->vw_full));
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(ms->kv_empty[s]));
+      if (lane == 0) mbar_arrive(bar(ms->v_empty[s]));
       crefl = cnewl;
     }
   } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ state image and phi(K)
+    // ------------------------------------------------------------ phi(K) and the state image
     const int q4 = warp & 3, row = q4 * 32 + lane;
     const uint32_t la = uint32_t(q4 * 32) << 16;
-    uint32_t kph = 0, ukc = 0;
-    for (int c = 0; c < nch; ++c) {
-      const int pz = c & 1;
-      // (1) image of S_{<c} at reference cref_c, then S rescaled to cnew_c
-      if (c >= 1 && !mbar_wait(bar(ms->s_done), (c - 1) & 1, abort_flag)) break;
-      if (!mbar_wait(bar(ms->meta_full[pz]), (c >> 1) & 1, abort_flag)) break;
-      if (c >= 1 && !mbar_wait(bar(ms->img_free), (c - 1) & 1, abort_flag)) break;
+    uint32_t ukc = 0;
+    // z_f as bf16 hi + lo parts in rows 0 and 1 of the K-major z operand (128-byte swizzle)
+    auto zrow_store = [&](float z) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(z);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(z - __bfloat162float(hi));
+      uint8_t* zb = gb + kC_ZROW + (row >> 6) * 2048 + (row & 7) * 2;
+      const int ch = (row & 63) >> 3;
+      *reinterpret_cast<__nv_bfloat16*>(zb + (ch << 4)) = hi;
+      *reinterpret_cast<__nv_bfloat16*>(zb + kRowB + ((ch ^ 1) << 4)) = lo;
+    };
+    // phi'(K_c) = a_j phi(k_j) into buffer c & 1, once P(c-2) and S(c-2) have read that buffer
+    // (S(c-2) is complete: the state image of chunk c-1 waited for it)
+    auto phi_k = [&](int c) -> bool {
+      if (c >= 2 && !mbar_wait(bar(ms->phik_free[c & 1]), ((c >> 1) - 1) & 1, abort_flag)) return false;
+      float aw = 1.f;
+      if (KIND == 0) {
+        if (!mbar_wait(bar(ms->meta_full[c & (kMeta - 1)]), (c / kMeta) & 1, abort_flag)) return false;
+        aw = sm->wk[c & (kMeta - 1)][row];
+      }
+      uint8_t* dstb = gb + kC_PHK + (c & 1) * kPhkB + row * kRowB;
+      for (int sl = 0; sl < NSL; ++sl) {
+        if (!mbar_wait(bar(ms->uk_full), ukc & 1, abort_flag)) return false;
+        ++ukc;
+        tc_fence_after();
+        // 4 groups of 16 angles, the next group's load in flight while the current is computed
+        auto grp16 = [&](const uint32_t(&u)[16], int gi) {
+          if (KIND == 0) {
+            // angle a -> features (2a, 2a+1) = (cos, sin): atom a / 32, 4 angles per 16 bytes
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int a = 16 * gi + 4 * q + e;
+                float sn, cs;
+                __sincosf(__uint_as_float(u[4 * q + e]), &sn, &cs);
+                pk[e] = g * NA + a < p.M ? pack_bf16x2(cs * aw, sn * aw) : 0u;
+              }
+              const int ch = (gi & 1) * 4 + q;
+              *reinterpret_cast<uint4*>(dstb + (gi >> 1) * kTileB + ((ch ^ (row & 7)) << 4)) =
+                  make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          } else {
+            // slice sl, angle a -> feature 64 sl + a: 8 features per 16 bytes
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                pk[e] = pack_bf16x2(fmaxf(__uint_as_float(u[8 * q + 2 * e]), 0.f),
+                                    fmaxf(__uint_as_float(u[8 * q + 2 * e + 1]), 0.f));
+              const int ch = 2 * gi + q;
+              *reinterpret_cast<uint4*>(dstb + sl * kTileB + ((ch ^ (row & 7)) << 4)) =
+                  make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        };
+        uint32_t ua[16], ub[16];
+        tmem_ld16(tmem + la + kT_B, ua);
+        tmem_wait_ld();
+#pragma unroll 1
+        for (int gi = 0; gi < 4; gi += 2) {
+          tmem_ld16(tmem + la + kT_B + 16 * (gi + 1), ub);
+          grp16(ua, gi);
+          tmem_wait_ld();
+          if (gi + 2 < 4) {
+            tmem_ld16(tmem + la + kT_B + 16 * (gi + 2), ua);
+          } else {
+            tc_fence_before();  // U_K is in registers: the next slice may overwrite it
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(ms->uk_free));
+          }
+          grp16(ub, gi + 1);
+          if (gi + 2 < 4) tmem_wait_ld();
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(ms->phik_full[c & 1]));
+      return true;
+    };
+    bool ok = nch == 0 || phi_k(0);
+    for (int c = 0; ok && c < nch; ++c) {
+      const int mb = c & (kMeta - 1);
+      // image of S_{<c} at reference cref_c, then S rescaled to cnew_c
+      if (c >= 1 && !(ok = mbar_wait(bar(ms->s_done), (c - 1) & 1, abort_flag))) break;
+      if (!(ok = mbar_wait(bar(ms->meta_full[mb]), (c / kMeta) & 1, abort_flag))) break;
+      if (c >= 1 && !(ok = mbar_wait(bar(ms->img_free), (c - 1) & 1, abort_flag))) break;
       tc_fence_after();
       uint8_t* img = gb + kC_IMG + row * kRowB;
       if (c == 0) {
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(img + (ch << 4)) = make_uint4(0u, 0u, 0u, 0u);
-        sm->z[row] = 0.f;
-        if (row == 0) sm->imgexp[pz] = 0.f;
+        zrow_store(0.f);
       } else {
         uint32_t a[32], b[32], zz[16];
         tmem_ld32(tmem + la + kT_S, a);
         tmem_ld32(tmem + la + kT_S + 32, b);
         tmem_ld16(tmem + la + kT_S + 64, zz);
         tmem_wait_ld();
-        float mx = 0.f;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(a[e])), fabsf(__uint_as_float(b[e]))));
-#pragma unroll
-        for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) sm->red[pz][q4] = mx;
-        if (!group_sync(bar(ms->ksync), kph, abort_flag)) break;
-        mx = fmaxf(fmaxf(sm->red[pz][0], sm->red[pz][1]), fmaxf(sm->red[pz][2], sm->red[pz][3]));
-        // power-of-two scale putting the largest |S| in [2^13, 2^14)
-        int e2 = 0;
-        if (mx > 1e-30f) {
-          const int ex = int((__float_as_uint(mx) >> 23) & 0xFF) - 127;
-          e2 = min(max(13 - ex, -120), 120);
-        }
-        const float sc = pow2i(e2);
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           const uint32_t* src = ch < 4 ? a + 8 * ch : b + 8 * (ch - 4);
           uint4 o;
-          o.x = pack_f16x2(__uint_as_float(src[0]) * sc, __uint_as_float(src[1]) * sc);
-          o.y = pack_f16x2(__uint_as_float(src[2]) * sc, __uint_as_float(src[3]) * sc);
-          o.z = pack_f16x2(__uint_as_float(src[4]) * sc, __uint_as_float(src[5]) * sc);
-          o.w = pack_f16x2(__uint_as_float(src[6]) * sc, __uint_as_float(src[7]) * sc);
+          o.x = pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1]));
+          o.y = pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3]));
+          o.z = pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5]));
+          o.w = pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7]));
           *reinterpret_cast<uint4*>(img + ((ch ^ (row & 7)) << 4)) = o;
         }
-        sm->z[row] = __uint_as_float(zz[0]);
-        if (row == 0) sm->imgexp[pz] = float(e2);
-        const float rho = ex2_approx(sm->crefl[pz] - sm->cnewl[pz]);
-        if (KIND == 0 && rho != 1.f) {
+        zrow_store(__uint_as_float(zz[0]));
+        if (KIND == 0) {
+          const float rho = ex2_approx(sm->crefl[mb] - sm->cnewl[mb]);
+          if (rho != 1.f) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            a[e] = __float_as_uint(__uint_as_float(a[e]) * rho);
-            b[e] = __float_as_uint(__uint_as_float(b[e]) * rho);
+            for (int e = 0; e < 32; ++e) {
+              a[e] = __float_as_uint(__uint_as_float(a[e]) * rho);
+              b[e] = __float_as_uint(__uint_as_float(b[e]) * rho);
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) zz[e] = __float_as_uint(__uint_as_float(zz[e]) * rho);
+            tmem_st32(tmem + la + kT_S, a);
+            tmem_st32(tmem + la + kT_S + 32, b);
+            tmem_st16(tmem + la + kT_S + 64, zz);
+            tmem_wait_st();
           }
-#pragma unroll
-          for (int e = 0; e < 16; ++e) zz[e] = __float_as_uint(__uint_as_float(zz[e]) * rho);
-          tmem_st32(tmem + la + kT_S, a);
-          tmem_st32(tmem + la + kT_S + 32, b);
-          tmem_st16(tmem + la + kT_S + 64, zz);
-          tmem_wait_st();
         }
       }
       fence_proxy_async_smem();
@@ -448,154 +585,109 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(ms->img_full));
         mbar_arrive(bar(ms->s_ready));
       }
-      // (2) phi(K_c) into shared memory (the buffer is free: S(c-1) has completed)
-      bool ok = true;
-      for (int sl = 0; sl < NSL; ++sl) {
-        if (!(ok = mbar_wait(bar(ms->uk_full), ukc & 1, abort_flag))) break;
-        ++ukc;
-        tc_fence_after();
-        uint32_t u0[32], u1[32];
-        tmem_ld32(tmem + la + kT_B, u0);
-        tmem_ld32(tmem + la + kT_B + 32, u1);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(ms->uk_free));
-        if (KIND == 0) {
-          // angle a -> features (2a, 2a+1) = (cos, sin); atom a / 32, 4 angles per 16 bytes
-#pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int a = 4 * q + e;
-              const float x = __uint_as_float(a < 32 ? u0[a] : u1[a - 32]);
-              float sn, cs;
-              __sincosf(x, &sn, &cs);
-              const bool live = g * NA + a < p.M;
-              pk[e] = live ? pack_f16x2(cs, sn) : 0u;
-            }
-            const int atom = q >> 3, ch = q & 7;
-            *reinterpret_cast<uint4*>(gb + kC_PHK + atom * kTileB + row * kRowB + ((ch ^ (row & 7)) << 4)) =
-                make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int a = 8 * q + 2 * e;
-              const float x0 = __uint_as_float(a < 32 ? u0[a] : u1[a - 32]);
-              const float x1 = __uint_as_float(a + 1 < 32 ? u0[a + 1] : u1[a + 1 - 32]);
-              pk[e] = pack_f16x2(fmaxf(x0, 0.f), fmaxf(x1, 0.f));
-            }
-            *reinterpret_cast<uint4*>(gb + kC_PHK + sl * kTileB + row * kRowB + ((q ^ (row & 7)) << 4)) =
-                make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          }
-        }
-      }
-      if (!ok) break;
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(ms->phik_full));
+      if (c + 1 < nch && !(ok = phi_k(c + 1))) break;
     }
-  } else if (warp >= 8) {
-    // ------------------------------------------------------------ phi(Q), P16, output
+  } else if (warp < 12) {
+    // ------------------------------------------------------------ phi(Q), P16, partial rows
     const int q4 = warp & 3, row = q4 * 32 + lane;
     const uint32_t la = uint32_t(q4 * 32) << 16;
     const int owner = q4 % G;
-    float dz_cur = 0.f, dz_prev = 0.f, di_cur = 0.f, di_prev = 0.f;
+    float di_cur = 0.f, di_prev = 0.f;
+    int pend = -1;  // chunk whose deposit is stored but not yet signalled
     // phi(Q_c): features into TMEM (in place over U_Q), and phi(q_i).z
     auto phi_q = [&](int c) -> bool {
       if (!mbar_wait(bar(ms->uq_full), c & 1, abort_flag)) return false;
-      if (!mbar_wait(bar(ms->img_full), c & 1, abort_flag)) return false;
       tc_fence_after();
-      float dz = 0.f;
       if (KIND == 0) {
-        uint32_t u0[32], u1[32];
-        tmem_ld32(tmem + la + kT_A, u0);
-        tmem_ld32(tmem + la + kT_A + 32, u1);
+        // 4 groups of 16 angles; angle a -> packed (cos, sin) in column a, in place. The next
+        // group's load is in flight while the current one is computed.
+        auto grp16 = [&](uint32_t(&u)[16], int gi) {
+#pragma unroll
+          for (int a = 0; a < 16; ++a) {
+            float sn, cs;
+            __sincosf(__uint_as_float(u[a]), &sn, &cs);
+            u[a] = pack_bf16x2(cs, sn);
+          }
+          tmem_st16(tmem + la + kT_A + 16 * gi, u);
+        };
+        uint32_t ua[16], ub[16];
+        tmem_ld16(tmem + la + kT_A, ua);
         tmem_wait_ld();
-#pragma unroll
-        for (int a = 0; a < 32; ++a) {
-          float sn, cs;
-          __sincosf(__uint_as_float(u0[a]), &sn, &cs);
-          const float2 zf = *reinterpret_cast<const float2*>(&sm->z[2 * a]);
-          dz = fmaf(cs, zf.x, fmaf(sn, zf.y, dz));
-          u0[a] = pack_f16x2(cs, sn);
+#pragma unroll 1
+        for (int gi = 0; gi < 4; gi += 2) {
+          tmem_ld16(tmem + la + kT_A + 16 * (gi + 1), ub);
+          grp16(ua, gi);
+          tmem_wait_ld();
+          if (gi + 2 < 4) tmem_ld16(tmem + la + kT_A + 16 * (gi + 2), ua);
+          grp16(ub, gi + 1);
+          tmem_wait_ld();
         }
-#pragma unroll
-        for (int a = 0; a < 32; ++a) {
-          float sn, cs;
-          __sincosf(__uint_as_float(u1[a]), &sn, &cs);
-          const float2 zf = *reinterpret_cast<const float2*>(&sm->z[64 + 2 * a]);
-          dz = fmaf(cs, zf.x, fmaf(sn, zf.y, dz));
-          u1[a] = pack_f16x2(cs, sn);
-        }
-        tmem_st32(tmem + la + kT_A, u0);
-        tmem_st32(tmem + la + kT_A + 32, u1);
       } else {
 #pragma unroll
-        for (int pc = 0; pc < 4; ++pc) {
+        for (int pc = 0; pc < NA / 32; ++pc) {
           uint32_t u[32], pk[16];
           tmem_ld32(tmem + la + kT_A + 32 * pc, u);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float x0 = fmaxf(__uint_as_float(u[2 * e]), 0.f), x1 = fmaxf(__uint_as_float(u[2 * e + 1]), 0.f);
-            const float2 zf = *reinterpret_cast<const float2*>(&sm->z[32 * pc + 2 * e]);
-            dz = fmaf(x0, zf.x, fmaf(x1, zf.y, dz));
-            pk[e] = pack_f16x2(x0, x1);
-          }
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(fmaxf(__uint_as_float(u[2 * e]), 0.f), fmaxf(__uint_as_float(u[2 * e + 1]), 0.f));
           tmem_st16(tmem + la + kT_A + 16 * pc, pk);
+        }
+        if (kHalfFeat) {  // features 64..127 of the block are zero
+          uint32_t zr[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) zr[e] = 0u;
+          tmem_st32(tmem + la + kT_A + 32, zr);
         }
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar(ms->phiq_full));
-        mbar_arrive(bar(ms->img_free));
-      }
-      dz_cur = dz;
+      if (lane == 0) mbar_arrive(bar(ms->phiq_full));
       return true;
     };
-    // P16 = weighted, masked P in bf16 (in place), and sum_j P16_ij
+    // P16 = masked P' in bf16 (in place; large-rise chunks also weight it), and sum_j P16_ij
     auto p16 = [&](int c) -> bool {
-      const int pz = c & 1;
+      const int mb = c & (kMeta - 1);
       if (!mbar_wait(bar(ms->p_full), c & 1, abort_flag)) return false;
-      if (!mbar_wait(bar(ms->meta_full[pz]), (c >> 1) & 1, abort_flag)) return false;
+      if (!mbar_wait(bar(ms->meta_full[mb]), (c / kMeta) & 1, abort_flag)) return false;
       tc_fence_after();
-      const float ri = sm->rl[pz][row];
+      const bool fb = KIND == 0 && sm->fb[mb];
+      const float ri = sm->rl[mb][row];
       const int rmax = q4 * 32 + 31;
       float di = 0.f;
 #pragma unroll 1
-      for (int pc = 0; pc < 4; ++pc) {
-        uint32_t pk[16];
-        if (32 * pc > rmax) {
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pk0[16], pk1[16];
+        if (64 * hf > rmax) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = 0u;
+          for (int e = 0; e < 16; ++e) pk0[e] = pk1[e] = 0u;
         } else {
-          uint32_t u[32];
-          tmem_ld32(tmem + la + kT_PR + 32 * pc, u);
+          uint32_t u0[32], u1[32];
+          tmem_ld32(tmem + la + kT_PR + 64 * hf, u0);
+          tmem_ld32(tmem + la + kT_PR + 64 * hf + 32, u1);
           tmem_wait_ld();
+          auto conv = [&](const uint32_t(&u)[32], uint32_t(&pk)[16], int j00) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int j0 = 32 * pc + 2 * e;
-            float x0 = __uint_as_float(u[2 * e]), x1 = __uint_as_float(u[2 * e + 1]);
-            if (KIND == 0) {
-              const float2 nn = *reinterpret_cast<const float2*>(&sm->n2l[pz][j0]);
-              x0 *= ex2_approx(nn.x - ri);
-              x1 *= ex2_approx(nn.y - ri);
+            for (int e = 0; e < 16; ++e) {
+              const int j0 = j00 + 2 * e;
+              float x0 = __uint_as_float(u[2 * e]), x1 = __uint_as_float(u[2 * e + 1]);
+              if (KIND == 0 && fb) {
+                const float2 rr = *reinterpret_cast<const float2*>(&sm->rl[mb][j0]);
+                x0 *= ex2_approx(rr.x - ri);
+                x1 *= ex2_approx(rr.y - ri);
+              }
+              x0 = j0 <= row ? x0 : 0.f;
+              x1 = j0 + 1 <= row ? x1 : 0.f;
+              pk[e] = pack_bf16x2(x0, x1);
+              di += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
             }
-            x0 = j0 <= row ? x0 : 0.f;
-            x1 = j0 + 1 <= row ? x1 : 0.f;
-            pk[e] = pack_bf16x2(x0, x1);
-            di += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
-          }
+          };
+          conv(u0, pk0, 64 * hf);
+          conv(u1, pk1, 64 * hf + 32);
         }
-        tmem_st16(tmem + la + kT_PR + 16 * pc, pk);
+        tmem_st16(tmem + la + kT_PR + 32 * hf, pk0);
+        tmem_st16(tmem + la + kT_PR + 32 * hf + 16, pk1);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -604,92 +696,133 @@ __global__ void __launch_bounds__(kThreads, 1)
       di_cur = di;
       return true;
     };
-    // output of chunk c: combine inter and intra, exchange partials, divide, store
-    auto output = [&](int c, float dz, float di) -> bool {
-      const int pz = c & 1;
+    // the partial row of chunk c: inter and intra combined at the row's reference; stored
+    // directly (G = 1) or deposited with the owner of the row. TMEM is released before the
+    // wait for the deposit slot, so the next chunk's P does not wait on the combiner.
+    auto output = [&](int c, float di) -> bool {
+      const int mb = c & (kMeta - 1);
       if (!mbar_wait(bar(ms->o_full), c & 1, abort_flag)) return false;
       tc_fence_after();
-      uint32_t in0[32], in1[32], it0[32], it1[32];
-      tmem_ld32(tmem + la + kT_IN, in0);
-      tmem_ld32(tmem + la + kT_IN + 32, in1);
-      tmem_ld32(tmem + la + kT_PR + 64, it0);
-      tmem_ld32(tmem + la + kT_PR + 96, it1);
-      tmem_wait_ld();
-      const float gfac = KIND == 0 ? ex2_approx(sm->crefl[pz] - sm->rl[pz][row]) : 1.f;
-      const float ffac = gfac * pow2i(-int(sm->imgexp[pz]));
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar(ms->pr_free));
-        mbar_arrive(bar(ms->meta_free[pz]));
-      }
-      float num[64];
+      const float ri = sm->rl[mb][row];
+      const float gfac = KIND == 0 ? ex2_approx(sm->crefl[mb] - ri) : 1.f;
+      const float rho = KIND == 0 && !sm->fb[mb] ? ex2_approx(sm->cnewl[mb] - ri) : 1.f;
+      float nm[64];
+      uint32_t dzh, dzl;
+      tmem_ld1(tmem + la + kT_IN + 64, dzh);
+      tmem_ld1(tmem + la + kT_IN + 65, dzl);
+      {
+        uint32_t in[32], it[32];
+        tmem_ld32(tmem + la + kT_IN, in);
+        tmem_ld32(tmem + la + kT_PR + 64, it);
+        tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        num[e] = fmaf(__uint_as_float(in0[e]), ffac, __uint_as_float(it0[e]));
-        num[32 + e] = fmaf(__uint_as_float(in1[e]), ffac, __uint_as_float(it1[e]));
+        for (int e = 0; e < 32; ++e) nm[e] = fmaf(__uint_as_float(in[e]), gfac, __uint_as_float(it[e]) * rho);
       }
-      float den = fmaf(dz, gfac, di);
-      if (G > 1) {
-        if (owner != g) {
-          // send this CTA's partial row to the owner of the rows
-          if (c >= 1 && !mbar_wait(bar(ms->recv_free[q4]), (c - 1) & 1, abort_flag)) return false;
-          const int qo = q4 / G, sidx = (g - owner + G) % G - 1;
-          const uint32_t dst =
-              mapa_shared(base + kC_RECV + ((qo * (G - 1) + sidx) * 32 + lane) * kRecvRowB, owner);
+      {
+        uint32_t in[32], it[32];
+        tmem_ld32(tmem + la + kT_IN + 32, in);
+        tmem_ld32(tmem + la + kT_PR + 96, it);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar(ms->pr_free));
+          mbar_arrive(bar(ms->meta_free[mb]));
+        }
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            st_dsmem_f4(dst + 16 * e, make_float4(num[4 * e], num[4 * e + 1], num[4 * e + 2], num[4 * e + 3]));
-          st_dsmem_f4(dst + 256, make_float4(den, 0.f, 0.f, 0.f));
-          mbar_arrive_remote(mapa_shared(smem_u32(&ms->recv_full[q4]), owner));
-          return true;
-        }
-        if (!mbar_wait_cluster(bar(ms->recv_full[q4]), c & 1, abort_flag)) return false;
-        const int qo = q4 / G;
-        for (int sidx = 0; sidx < G - 1; ++sidx) {
-          const float* src =
-              reinterpret_cast<const float*>(gb + kC_RECV + ((qo * (G - 1) + sidx) * 32 + lane) * kRecvRowB);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float4 x = *reinterpret_cast<const float4*>(src + 4 * e);
-            num[4 * e] += x.x;
-            num[4 * e + 1] += x.y;
-            num[4 * e + 2] += x.z;
-            num[4 * e + 3] += x.w;
-          }
-          den += src[64];
-        }
-        // the received rows are consumed: let each sender reuse its slot
-        for (int sidx = 0; sidx < G - 1; ++sidx) {
-          const int sender = (owner + 1 + sidx) % G;
-          mbar_arrive_remote(mapa_shared(smem_u32(&ms->recv_free[q4]), sender));
-        }
+        for (int e = 0; e < 32; ++e) nm[32 + e] = fmaf(__uint_as_float(in[e]), gfac, __uint_as_float(it[e]) * rho);
       }
-      const int token = c * kTile + row;
-      if (token < L) {
-        const float inv = den != 0.f ? 1.f / den : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)bh * L + token) * kD);
+      const float den = fmaf(__uint_as_float(dzh) + __uint_as_float(dzl), gfac, di * rho);
+      if (G == 1) {
+        const int token = c * kTile + row;
+        if (token < L) {
+          const float inv = den != 0.f ? 1.f / den : 0.f;
+          uint4* o = reinterpret_cast<uint4*>(out + ((size_t)bh * L + token) * kD);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          uint4 o;
-          o.x = pack_bf16x2(num[8 * q] * inv, num[8 * q + 1] * inv);
-          o.y = pack_bf16x2(num[8 * q + 2] * inv, num[8 * q + 3] * inv);
-          o.z = pack_bf16x2(num[8 * q + 4] * inv, num[8 * q + 5] * inv);
-          o.w = pack_bf16x2(num[8 * q + 6] * inv, num[8 * q + 7] * inv);
-          dst[q] = o;
+          for (int q = 0; q < 8; ++q)
+            o[q] = make_uint4(pack_bf16x2(nm[8 * q] * inv, nm[8 * q + 1] * inv),
+                              pack_bf16x2(nm[8 * q + 2] * inv, nm[8 * q + 3] * inv),
+                              pack_bf16x2(nm[8 * q + 4] * inv, nm[8 * q + 5] * inv),
+                              pack_bf16x2(nm[8 * q + 6] * inv, nm[8 * q + 7] * inv));
         }
+        return true;
       }
+      // the previous chunk's deposit: its release no longer waits for stores in flight
+      if (pend >= 0) {
+        mbar_arrive_remote(mapa_shared(smem_u32(&ms->recv_full[q4][pend & 1]), owner));
+        pend = -1;
+      }
+      // deposit buffer c & 1: free once the owner has combined chunk c - 2
+      const int pb = c & 1;
+      if (c >= 2 && !mbar_wait(bar(ms->recv_free[q4][pb]), ((c >> 1) - 1) & 1, abort_flag)) return false;
+      const int qo = q4 / G;
+      const uint32_t dst =
+          mapa_shared(base + kC_RECV + pb * kRecvBufB + ((qo * G + g) * 32 + lane) * kRecvRowB, owner);
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        st_dsmem_f4(dst + 16 * e,
+                    make_float4(__uint_as_float(pack_bf16x2(nm[8 * e], nm[8 * e + 1])),
+                                __uint_as_float(pack_bf16x2(nm[8 * e + 2], nm[8 * e + 3])),
+                                __uint_as_float(pack_bf16x2(nm[8 * e + 4], nm[8 * e + 5])),
+                                __uint_as_float(pack_bf16x2(nm[8 * e + 6], nm[8 * e + 7]))));
+      st_dsmem_f4(dst + 128, make_float4(den, 0.f, 0.f, 0.f));
+      pend = c;  // signalled at the next deposit (or after the last), once the stores have landed
       return true;
     };
     bool ok = true;
     for (int c = 0; ok && c < nch; ++c) {
       if (!(ok = phi_q(c))) break;
-      if (c >= 1 && !(ok = output(c - 1, dz_prev, di_prev))) break;
+      if (c >= 1 && !(ok = output(c - 1, di_prev))) break;
       if (!(ok = p16(c))) break;
-      dz_prev = dz_cur;
       di_prev = di_cur;
     }
-    if (ok && nch > 0) output(nch - 1, dz_prev, di_prev);
+    if (ok && nch > 0) output(nch - 1, di_prev);
+    if (G > 1 && pend >= 0) mbar_arrive_remote(mapa_shared(smem_u32(&ms->recv_full[q4][pend & 1]), owner));
+  } else if (G > 1) {
+    // ------------------------------------------------------------ combiner (warp 12)
+    // Rows 32 q .. 32 q + 31 (q % G == g) of every chunk: the G partial rows, summed in CTA
+    // order, divided and stored; every depositor may reuse its slot once they are read.
+    bool ok = true;
+    for (int c = 0; ok && c < nch; ++c) {
+      const int pb = c & 1;
+      for (int q = g; q < 4; q += G) {
+        if (!(ok = mbar_wait_cluster(bar(ms->recv_full[q][pb]), (c >> 1) & 1, abort_flag))) break;
+        const int qo = q / G;
+        const uint8_t* src0 = gb + kC_RECV + pb * kRecvBufB + ((qo * G) * 32 + lane) * kRecvRowB;
+        float acc[64], den = 0.f;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) acc[e] = 0.f;
+        for (int s = 0; s < G; ++s) {
+          const uint8_t* src = src0 + s * 32 * kRecvRowB;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint4 x = *reinterpret_cast<const uint4*>(src + 16 * e);
+            const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              acc[8 * e + 2 * t] += __uint_as_float(w4[t] << 16);
+              acc[8 * e + 2 * t + 1] += __uint_as_float(w4[t] & 0xFFFF0000u);
+            }
+          }
+          den += *reinterpret_cast<const float*>(src + 128);
+        }
+        // the slots are in registers: release them (one fence, then relaxed arrives that do not
+        // wait for one another) before the global stores
+        fence_acq_rel_cluster();
+        for (int s = 0; s < G; ++s) mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&ms->recv_free[q][pb]), s));
+        const float inv = den != 0.f ? 1.f / den : 0.f;
+        const int token = c * kTile + q * 32 + lane;
+        if (token < L) {
+          uint4* o = reinterpret_cast<uint4*>(out + ((size_t)bh * L + token) * kD);
+#pragma unroll
+          for (int q8 = 0; q8 < 8; ++q8)
+            o[q8] = make_uint4(pack_bf16x2(acc[8 * q8] * inv, acc[8 * q8 + 1] * inv),
+                               pack_bf16x2(acc[8 * q8 + 2] * inv, acc[8 * q8 + 3] * inv),
+                               pack_bf16x2(acc[8 * q8 + 4] * inv, acc[8 * q8 + 5] * inv),
+                               pack_bf16x2(acc[8 * q8 + 6] * inv, acc[8 * q8 + 7] * inv));
+        }
+      }
+    }
   }
 
   // ---------------------------------------------------------------- teardown

@@ -112,6 +112,13 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
 
+// Relaxed variant: no ordering of its own. Precede it with fence_acq_rel_cluster() when the
+// waiter must see this thread's earlier accesses as done.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+
 // Bounded barrier among the `count` threads an mbarrier was initialised with: arrive, then
 // wait for the phase to complete. `phase` is this thread's running phase bit.
 __device__ __forceinline__ bool group_sync(uint32_t bar, uint32_t& phase, volatile int* abort) {
