@@ -35,6 +35,29 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 METRIC = "FAVOR fwd tokens/s (B·H·L/s) at L=4096,d=64,M=256; % of tensor/HBM roofline"
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of each variant's kernel
+# at this workload, from one ncu capture (profiles/), with the SHA-1 of the kernel sources the
+# capture was taken with. A value whose sources have changed since is reported as null.
+TRAFFIC = {
+    "trig_bidir": (51576576, "7b128e47050d0b36c57044a198561c2e64e28886"),
+    "relu_bidir": (51480064, "7b128e47050d0b36c57044a198561c2e64e28886"),
+    "trig_causal": (51230464, "7b128e47050d0b36c57044a198561c2e64e28886"),
+    "relu_causal": (51767296, "7b128e47050d0b36c57044a198561c2e64e28886"),
+}
+KERNEL_SOURCES = ["linear_kernelized_attention_b200/csrc/ptx.cuh",
+                  "linear_kernelized_attention_b200/csrc/kernel_bidir.cuh",
+                  "linear_kernelized_attention_b200/csrc/kernel_causal.cuh"]
+
+
+def kernel_sources_sha():
+    import hashlib
+    h = hashlib.sha1()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
 def flops_per_token(d, M, kind):
     F = 2 * M if kind == 0 else M
     return 4 * d * M + 4 * F * (d + 1)
@@ -280,8 +303,10 @@ def main():
     flops = flops_per_token(d, M, kind) * B * H * L
     achieved = flops / (per_variant[dom] * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    tr = TRAFFIC.get(dom)
+    traffic = tr[0] if tr and tr[1] == kernel_sources_sha() else None
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": None, "kernel": dom,
+            "frac": achieved / peak, "traffic": traffic, "kernel": dom,
             "peak_source": f"{peak_src} bf16 burst", "ms_per_launch": per_variant[dom]}
 
     # end to end through the host-buffer C ABI entry (pinned host memory, copies timed)

@@ -668,6 +668,15 @@ __global__ void __launch_bounds__(kThreadsC, 1)
           tmem_ld32(tmem + la + kT_PR + 64 * hf + 32, u1);
           tmem_wait_ld();
           auto conv = [&](const uint32_t(&u)[32], uint32_t(&pk)[16], int j00) {
+            if (!(KIND == 0 && fb) && j00 + 31 <= q4 * 32) {
+              // every key of this piece precedes every row of the warp: no mask, no weight
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                pk[e] = pack_bf16x2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
+                di += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+              }
+              return;
+            }
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int j0 = j00 + 2 * e;
