@@ -474,7 +474,7 @@ __global__ void __launch_bounds__(kThreadsC, 1)
         if (!mbar_wait(bar(ms->uk_full), ukc & 1, abort_flag)) return false;
         ++ukc;
         tc_fence_after();
-        // 4 groups of 16 angles, the next group's load in flight while the current is computed
+        // 4 groups of 16 angles
         auto grp16 = [&](const uint32_t(&u)[16], int gi) {
           if (KIND == 0) {
             // angle a -> features (2a, 2a+1) = (cos, sin): atom a / 32, 4 angles per 16 bytes
@@ -507,23 +507,17 @@ __global__ void __launch_bounds__(kThreadsC, 1)
             }
           }
         };
-        uint32_t ua[16], ub[16];
-        tmem_ld16(tmem + la + kT_B, ua);
-        tmem_wait_ld();
 #pragma unroll 1
-        for (int gi = 0; gi < 4; gi += 2) {
-          tmem_ld16(tmem + la + kT_B + 16 * (gi + 1), ub);
-          grp16(ua, gi);
+        for (int gi = 0; gi < 4; ++gi) {
+          uint32_t u[16];
+          tmem_ld16(tmem + la + kT_B + 16 * gi, u);
           tmem_wait_ld();
-          if (gi + 2 < 4) {
-            tmem_ld16(tmem + la + kT_B + 16 * (gi + 2), ua);
-          } else {
+          if (gi == 3) {
             tc_fence_before();  // U_K is in registers: the next slice may overwrite it
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(ms->uk_free));
           }
-          grp16(ub, gi + 1);
-          if (gi + 2 < 4) tmem_wait_ld();
+          grp16(u, gi);
         }
       }
       fence_proxy_async_smem();
@@ -599,8 +593,7 @@ __global__ void __launch_bounds__(kThreadsC, 1)
       if (!mbar_wait(bar(ms->uq_full), c & 1, abort_flag)) return false;
       tc_fence_after();
       if (KIND == 0) {
-        // 4 groups of 16 angles; angle a -> packed (cos, sin) in column a, in place. The next
-        // group's load is in flight while the current one is computed.
+        // 4 groups of 16 angles; angle a -> packed (cos, sin) in column a, in place
         auto grp16 = [&](uint32_t(&u)[16], int gi) {
 #pragma unroll
           for (int a = 0; a < 16; ++a) {
@@ -610,17 +603,12 @@ __global__ void __launch_bounds__(kThreadsC, 1)
           }
           tmem_st16(tmem + la + kT_A + 16 * gi, u);
         };
-        uint32_t ua[16], ub[16];
-        tmem_ld16(tmem + la + kT_A, ua);
-        tmem_wait_ld();
 #pragma unroll 1
-        for (int gi = 0; gi < 4; gi += 2) {
-          tmem_ld16(tmem + la + kT_A + 16 * (gi + 1), ub);
-          grp16(ua, gi);
+        for (int gi = 0; gi < 4; ++gi) {
+          uint32_t u[16];
+          tmem_ld16(tmem + la + kT_A + 16 * gi, u);
           tmem_wait_ld();
-          if (gi + 2 < 4) tmem_ld16(tmem + la + kT_A + 16 * (gi + 2), ua);
-          grp16(ub, gi + 1);
-          tmem_wait_ld();
+          grp16(u, gi);
         }
       } else {
 #pragma unroll
@@ -656,47 +644,34 @@ __global__ void __launch_bounds__(kThreadsC, 1)
       const float ri = sm->rl[mb][row];
       const int rmax = q4 * 32 + 31;
       float di = 0.f;
+      // one 32-key piece per iteration, in place: piece pc (columns 32 pc ..) becomes 16 packed
+      // columns at 16 pc, which the earlier pieces have already read
 #pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t pk0[16], pk1[16];
-        if (64 * hf > rmax) {
+      for (int pc = 0; pc < 4; ++pc) {
+        uint32_t pk[16];
+        if (32 * pc > rmax) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) pk0[e] = pk1[e] = 0u;
+          for (int e = 0; e < 16; ++e) pk[e] = 0u;
         } else {
-          uint32_t u0[32], u1[32];
-          tmem_ld32(tmem + la + kT_PR + 64 * hf, u0);
-          tmem_ld32(tmem + la + kT_PR + 64 * hf + 32, u1);
+          uint32_t u[32];
+          tmem_ld32(tmem + la + kT_PR + 32 * pc, u);
           tmem_wait_ld();
-          auto conv = [&](const uint32_t(&u)[32], uint32_t(&pk)[16], int j00) {
-            if (!(KIND == 0 && fb) && j00 + 31 <= q4 * 32) {
-              // every key of this piece precedes every row of the warp: no mask, no weight
 #pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                pk[e] = pack_bf16x2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
-                di += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
-              }
-              return;
+          for (int e = 0; e < 16; ++e) {
+            const int j0 = 32 * pc + 2 * e;
+            float x0 = __uint_as_float(u[2 * e]), x1 = __uint_as_float(u[2 * e + 1]);
+            if (KIND == 0 && fb) {
+              const float2 rr = *reinterpret_cast<const float2*>(&sm->rl[mb][j0]);
+              x0 *= ex2_approx(rr.x - ri);
+              x1 *= ex2_approx(rr.y - ri);
             }
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int j0 = j00 + 2 * e;
-              float x0 = __uint_as_float(u[2 * e]), x1 = __uint_as_float(u[2 * e + 1]);
-              if (KIND == 0 && fb) {
-                const float2 rr = *reinterpret_cast<const float2*>(&sm->rl[mb][j0]);
-                x0 *= ex2_approx(rr.x - ri);
-                x1 *= ex2_approx(rr.y - ri);
-              }
-              x0 = j0 <= row ? x0 : 0.f;
-              x1 = j0 + 1 <= row ? x1 : 0.f;
-              pk[e] = pack_bf16x2(x0, x1);
-              di += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
-            }
-          };
-          conv(u0, pk0, 64 * hf);
-          conv(u1, pk1, 64 * hf + 32);
+            x0 = j0 <= row ? x0 : 0.f;
+            x1 = j0 + 1 <= row ? x1 : 0.f;
+            pk[e] = pack_bf16x2(x0, x1);
+            di += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+          }
         }
-        tmem_st16(tmem + la + kT_PR + 32 * hf, pk0);
-        tmem_st16(tmem + la + kT_PR + 32 * hf + 16, pk1);
+        tmem_st16(tmem + la + kT_PR + 16 * pc, pk);
       }
       tmem_wait_st();
       tc_fence_before();

@@ -62,11 +62,11 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait until the phase with the given parity has completed. Bounded: returns false after
-// kWaitLimitCycles (or at once if *abort is set) and records FAVOR_ERR_TIMEOUT.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
-                                          volatile int* abort = nullptr,
-                                          long long limit = kWaitLimitCycles) {
-  if (mbar_try_wait(bar, parity)) return true;
+// `limit` cycles (or at once if *abort is set) and records FAVOR_ERR_TIMEOUT. The first test is
+// inline; the spin loop is one out-of-line function shared by every call site, which keeps the
+// kernels' executed code small.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort,
+                                            long long limit) {
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -77,6 +77,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          volatile int* abort = nullptr,
+                                          long long limit = kWaitLimitCycles) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort, limit);
 }
 
 // Cluster-scope acquire variant of the bounded wait, for barriers that other CTAs of the
@@ -92,7 +98,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort) {
+__device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
