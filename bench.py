@@ -10,9 +10,10 @@ rotating input sets (268 MB in total, more than 2x the 126 MB L2) keep every ste
 
 N > 1 is launched by torch.distributed.run. Each rank runs its own batch on its own GPU (the
 heads are independent), so per-GPU work is fixed ("weak" scaling) and there is no data-path
-collective. Timing: each (input set, variant) launch is captured once in a CUDA graph; the
-timed region replays them on one stream with CUDA events around every launch, barrier +
-synchronize on both sides, max over ranks.
+collective. Timing: one CUDA graph per input set holds a step (the four variants back to back);
+the timed region replays K of them between CUDA events on the launching stream, barrier +
+synchronize on both sides, max over ranks. Per-kernel launch durations (for the roofline) come
+from each variant's own graph, replayed between CUDA events in the same run.
 """
 from __future__ import annotations
 
@@ -239,37 +240,33 @@ def main():
         _, kind, causal = variants[j]
         F.favor_attention(q, k, v, omega, out=outs[s][j], feature_kind=kind, causal=causal, stream=st)
 
-    # eager warm-up (first-call set-up happens here), then one CUDA graph per (input set,
-    # variant): a replay launches exactly one kernel, without the per-call host work
+    # eager warm-up (first-call set-up happens here); the graphs below then launch the kernels
+    # without the per-call host work
     for i in range(args.warmup):
         for j in range(len(variants)):
             launch(i % N_SETS, j, stream)
     torch.cuda.synchronize()
     if F.favor_sync_status(stream) != 0:
         raise RuntimeError("device status not OK after warm-up")
-    graphs = [[torch.cuda.CUDAGraph() for _ in variants] for _ in range(N_SETS)]
+    # one CUDA graph per input set holding the four variants back to back (a step), and one per
+    # variant holding its launch on each input set (for the per-kernel durations)
+    step_graphs = [torch.cuda.CUDAGraph() for _ in range(N_SETS)]
     for s in range(N_SETS):
-        for j in range(len(variants)):
-            with torch.cuda.graph(graphs[s][j], stream=stream):
+        with torch.cuda.graph(step_graphs[s], stream=stream):
+            for j in range(len(variants)):
+                launch(s, j, stream)
+    var_graphs = [torch.cuda.CUDAGraph() for _ in variants]
+    for j in range(len(variants)):
+        with torch.cuda.graph(var_graphs[j], stream=stream):
+            for s in range(N_SETS):
                 launch(s, j, stream)
     torch.cuda.synchronize()
-
-    def step(i, ev=None):
-        for j in range(len(variants)):
-            if ev is not None:
-                ev[j][0].record(stream)
-            graphs[i % N_SETS][j].replay()
-            if ev is not None:
-                ev[j][1].record(stream)
-
     for i in range(args.warmup):
-        step(i)
+        step_graphs[i % N_SETS].replay()
     torch.cuda.synchronize()
 
     clocks = ClockSampler(local)
     clocks.start()
-    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-            for _ in variants] for _ in range(args.steps)]
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
@@ -277,7 +274,7 @@ def main():
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(args.steps):
-        step(i, evs[i])
+        step_graphs[i % N_SETS].replay()
     e1.record(stream)
     torch.cuda.synchronize()
     clocks.active.clear()
@@ -291,8 +288,18 @@ def main():
         ms = float(t.item())
     if F.favor_sync_status(stream) != 0:
         raise RuntimeError("device status not OK after the timed region")
-    per_variant = {name: float(np.mean([evs[i][j][0].elapsed_time(evs[i][j][1]) for i in range(args.steps)]))
-                   for j, (name, _, _) in enumerate(variants)}
+    # per-kernel average launch duration: each variant's graph (one launch per input set, back to
+    # back) replayed between CUDA events on the launching stream
+    reps = max(1, min(args.steps, 200) // N_SETS)
+    per_variant = {}
+    for j, (name, _, _) in enumerate(variants):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            var_graphs[j].replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        per_variant[name] = a.elapsed_time(b) / (reps * N_SETS)
     tokens_step = len(variants) * B * H * L
     value = world * tokens_step / (ms * 1e-3)
 
@@ -352,7 +359,7 @@ def main():
             "gpu_launches": args.steps * len(variants), "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)
-    del graphs
+    del step_graphs, var_graphs
     if dist:
         dist.barrier()
         dist.destroy_process_group()

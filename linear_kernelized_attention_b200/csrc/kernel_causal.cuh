@@ -656,17 +656,17 @@ __global__ void __launch_bounds__(kThreadsC, 1)
           uint32_t u[32];
           tmem_ld32(tmem + la + kT_PR + 32 * pc, u);
           tmem_wait_ld();
+          if (KIND == 0 && fb) {  // large-rise chunk: exact weights exp(R_j - R_i) (a separate
+                                  // loop, so the usual path stays compact)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              u[e] = __float_as_uint(__uint_as_float(u[e]) * ex2_approx(sm->rl[mb][32 * pc + e] - ri));
+          }
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int j0 = 32 * pc + 2 * e;
-            float x0 = __uint_as_float(u[2 * e]), x1 = __uint_as_float(u[2 * e + 1]);
-            if (KIND == 0 && fb) {
-              const float2 rr = *reinterpret_cast<const float2*>(&sm->rl[mb][j0]);
-              x0 *= ex2_approx(rr.x - ri);
-              x1 *= ex2_approx(rr.y - ri);
-            }
-            x0 = j0 <= row ? x0 : 0.f;
-            x1 = j0 + 1 <= row ? x1 : 0.f;
+            const float x0 = j0 <= row ? __uint_as_float(u[2 * e]) : 0.f;
+            const float x1 = j0 + 1 <= row ? __uint_as_float(u[2 * e + 1]) : 0.f;
             pk[e] = pack_bf16x2(x0, x1);
             di += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
           }
