@@ -40,10 +40,10 @@ METRIC = "FAVOR fwd tokens/s (B·H·L/s) at L=4096,d=64,M=256; % of tensor/HBM r
 # at this workload, from one ncu capture (profiles/), with the SHA-1 of the kernel sources the
 # capture was taken with. A value whose sources have changed since is reported as null.
 TRAFFIC = {
-    "trig_bidir": (51576576, "7b128e47050d0b36c57044a198561c2e64e28886"),
-    "relu_bidir": (51480064, "7b128e47050d0b36c57044a198561c2e64e28886"),
-    "trig_causal": (51230464, "7b128e47050d0b36c57044a198561c2e64e28886"),
-    "relu_causal": (51767296, "7b128e47050d0b36c57044a198561c2e64e28886"),
+    "trig_bidir": (51392000, "f95d0ce2faf5715457f577f8bcf35140ab04a556"),
+    "relu_bidir": (51413248, "f95d0ce2faf5715457f577f8bcf35140ab04a556"),
+    "trig_causal": (51099392, "f95d0ce2faf5715457f577f8bcf35140ab04a556"),
+    "relu_causal": (51088640, "f95d0ce2faf5715457f577f8bcf35140ab04a556"),
 }
 KERNEL_SOURCES = ["linear_kernelized_attention_b200/csrc/ptx.cuh",
                   "linear_kernelized_attention_b200/csrc/kernel_bidir.cuh",
