@@ -59,6 +59,18 @@ def kernel_sources_sha():
     return h.hexdigest()
 
 
+def max_over_ranks(x, device=None):
+    """Max of a per-rank number over all ranks of the default process group (the number itself
+    when torch.distributed is not initialised). Every rank must call it."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def flops_per_token(d, M, kind):
     F = 2 * M if kind == 0 else M
     return 4 * d * M + 4 * F * (d + 1)
@@ -281,11 +293,7 @@ def main():
     if dist:
         dist.barrier()
     clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
     if F.favor_sync_status(stream) != 0:
         raise RuntimeError("device status not OK after the timed region")
     # per-kernel average launch duration: each variant's graph (one launch per input set, back to
@@ -330,11 +338,7 @@ def main():
     for _ in range(n_e2e):
         for _, kind, causal in variants:
             F.favor_attention_host(hq, hk, hv, hom, hout, feature_kind=kind, causal=causal)
-    e2e_s = (time.perf_counter() - t0) / n_e2e
-    if dist:
-        t = torch.tensor([e2e_s], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
+    e2e_s = max_over_ranks((time.perf_counter() - t0) / n_e2e, dev)
     nx = B * H * L * d * 2
     e2e = {"value": world * tokens_step / e2e_s, "unit": "tokens/s",
            "h2d_bytes_per_step": len(variants) * (3 * nx + H * M * d * 2),

@@ -34,8 +34,10 @@
  * launch errors. Errors from inside a kernel surface at the next synchronisation.
  * favor_sync_status() synchronises the stream and returns the device-side status word.
  *
- * Scratch. Calls that need scratch take it from cudaMallocAsync on `stream` and release it
- * with cudaFreeAsync on the same stream.
+ * Scratch. The bf16 path needs none (cross-CTA sums travel through distributed shared memory).
+ * favor_attention_f32 and favor_attention_host take scratch from a library-owned stream-ordered
+ * pool on `stream` and release it on the same stream; favor_attention_f32_noalloc uses a static
+ * device array instead.
  *
  * Errors. Negative favor_status codes. On an error nothing is launched and no output is
  * written.
@@ -70,13 +72,18 @@ typedef enum {
 /*
  * bf16 forward pass: the tensor-core path.
  * q, k, v, omega, out: device pointers to __nv_bfloat16, 16-byte aligned, layouts above.
- * Supported: d in {32, 64}; M a multiple of 16 with 16 <= M <= 256 (trig) or <= 512 (relu);
- * L >= 1 (ragged tails are masked); B*H <= 65535.
- * Arithmetic: Q Omega^T and K Omega^T on tensor cores (bf16 in, fp32 accumulate).
- * Features in fp32 registers. phi(K) is rounded to bf16 for phi(K)^T [V|1] (fp32 accumulate).
- * The state is rounded to fp16 under a power-of-two scale, phi(Q) to fp16, and
- * phi(Q) S is accumulated in fp32. The normaliser division is in fp32, and the result is
- * rounded once to bf16.
+ * Supported: d = 64; M a multiple of 16 with 16 <= M <= 256 (trig) or <= 512 (relu);
+ * L >= 1 (ragged tails are masked); B*H <= 524280 (bidirectional) or B*H*ceil(M/64) (trig, and
+ * relu with M <= 256) / B*H*ceil(M/128) (relu, M > 256) < 2^31 (causal). Other shapes return
+ * FAVOR_ERR_UNSUPPORTED and launch nothing.
+ * Arithmetic: Q Omega^T and K Omega^T on tensor cores (bf16 in, fp32 accumulate); features in
+ * fp32 registers; every product on tensor cores accumulates in fp32.
+ *   Bidirectional: phi(K) is rounded to bf16 for phi(K)^T [V|1]; the state is rounded to fp16
+ *   under a power-of-two scale and phi(Q) to fp16 for phi(Q) S.
+ *   Causal (128-token chunks): phi(K) (carrying its stabiliser weight), phi(Q), the masked
+ *   intra-chunk scores and the state image are rounded to bf16; the state's normaliser column
+ *   enters phi(Q).z as a bf16 hi + lo pair; the intra-chunk denominator is summed in fp32.
+ * The normaliser division is in fp32, and the result is rounded once to bf16.
  * A zero denominator gives a zero output row.
  */
 int favor_attention(const void* q, const void* k, const void* v, const void* omega, void* out,
@@ -84,9 +91,10 @@ int favor_attention(const void* q, const void* k, const void* v, const void* ome
                     void* stream);
 
 /*
- * As favor_attention, with an explicit causal chunk length (64 or 128 tokens; 0 picks
- * the default). The chunk changes how the prefix sum is blocked, not its value.
- * Ignored when causal == 0.
+ * As favor_attention, with an explicit causal chunk length. The chunk changes how the prefix
+ * sum is blocked, not its value. The tensor-core kernel scans 128-token chunks: chunk 0 (the
+ * default) or 128; any other value returns FAVOR_ERR_UNSUPPORTED when causal != 0. Ignored when
+ * causal == 0.
  */
 int favor_attention_chunked(const void* q, const void* k, const void* v, const void* omega,
                             void* out, int B, int H, int L, int d, int M, int feature_kind,
