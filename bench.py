@@ -201,6 +201,57 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_lsweep(args):
+    """Throughput against sequence length at B=1, H=16, d=64, M=256 (trig, bidirectional and
+    causal), L = 4096 .. 65536: one JSON line per (L, variant). Constant tokens/s across L is
+    linear scaling. Rotating input sets keep every point's reads above twice the L2 size."""
+    import numpy as np
+    import torch
+
+    import favor_inputs as fi
+    import linear_kernelized_attention_b200 as F
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    B, H, d, M = 1, 16, 64, 256
+    G, R = fi.orf_gaussians(H, M, d, seed=0)
+    omega = F.favor_orf_omega(torch.from_numpy(G).to(dev), torch.from_numpy(R).to(dev), M, dtype=torch.bfloat16)
+    for L in (4096, 8192, 16384, 32768, 65536):
+        nbytes = 3 * B * H * L * d * 2
+        nsets = max(1, int(np.ceil(2 * 126e6 / nbytes)))
+        sets = []
+        for si in range(nsets):
+            q, k, v = fi.qkv(B, H, L, d, seed=si)
+            sets.append([fi.round_to(x, "bf16").to(dev) for x in (q, k, v)])
+        out = torch.empty_like(sets[0][0])
+        for causal in (False, True):
+            for si in range(nsets):
+                F.favor_attention(*sets[si], omega, out=out, feature_kind=0, causal=causal, stream=stream)
+            torch.cuda.synchronize()
+            if F.favor_sync_status(stream) != 0:
+                raise RuntimeError("device status not OK")
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for si in range(nsets):
+                    F.favor_attention(*sets[si], omega, out=out, feature_kind=0, causal=causal, stream=stream)
+            g.replay()
+            torch.cuda.synchronize()
+            reps = max(3, int(64 / nsets))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            us = 1e3 * a.elapsed_time(b) / (reps * nsets)
+            print(json.dumps({"lsweep": True, "L": L, "B": B, "H": H, "d": d, "M": M,
+                              "variant": "trig_causal" if causal else "trig_bidir", "us_per_launch": us,
+                              "tokens_per_s": B * H * L / (us * 1e-6), "input_sets": nsets}), flush=True)
+            del g
+        del sets
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -208,7 +259,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lsweep", action="store_true",
+                    help="throughput against L (B=1, H=16, trig) instead of the bench line")
     args = ap.parse_args()
+    if args.lsweep:
+        return run_lsweep(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
