@@ -47,6 +47,25 @@ def test_causal_relu_512_features():
     check_rows(g, ref, cond, TOL_BF16, U_BF16, "causal relu M=512")
 
 
+def test_causal_relu_384_features():
+    # ReLU M = 384: 128-angle blocks, 3 rounded up to G = 4 (one block is all padding)
+    c = Case(1, 2, 300, 64, 384, seed=12)
+    g = _run(c, 1).reshape(2, 300, 64)
+    ref, cond, _ = c.oracle(1, True)
+    check_rows(g, ref, cond, TOL_BF16, U_BF16, "causal relu M=384")
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+def test_causal_more_heads_than_sms(kind):
+    # B*H = 160 heads, 2 CTAs each: several waves of clusters
+    c = Case(2, 80, 200, 64, 128, seed=13)
+    g = _run(c, kind).reshape(160, 200, 64)
+    heads = [(0, 0), (0, 79), (1, 40), (1, 79)]
+    ref, cond, _ = c.oracle(kind, True, heads=heads)
+    sel = np.stack([g[b * 80 + h] for b, h in heads])
+    check_rows(sel, ref, cond, TOL_BF16, U_BF16, f"causal many heads kind={kind}")
+
+
 def test_causal_first_row_is_v0():
     # row 0 attends to key 0 only, so out_0 = v_0 for either map (non-zero denominator)
     c = Case(1, 2, 256, 64, 128, seed=21)
