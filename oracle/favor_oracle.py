@@ -299,6 +299,29 @@ def favor_rows_head(q, k, v, Om, kind, causal, rows):
     return out
 
 
+# ---------------------------------------------------------------- decode: one token per call
+def favor_decode_state(M, dv, kind):
+    """An empty carried state (S [F, dv], z [F]) for one head; F = 2M (trig) or M (ReLU)."""
+    F = 2 * M if kind == TRIG else M
+    return np.zeros((F, dv)), np.zeros(F)
+
+
+def favor_decode_step_head(S, z, q, k, v, Om, kind):
+    """One causal step for one head with a carried state. S and z are updated in place.
+
+    [EXPL, 核心机制]: the causal prefix sum of phi(k_j) v_j^T (and of phi(k_j) for the
+    normaliser) over j <= i, read by phi(q_i). Token i's key and value enter the state
+    before its query reads it, so starting from an empty state the i-th call returns
+    causal row i.
+    """
+    fk = phi(k[None, :], Om, kind)[0]
+    fq = phi(q[None, :], Om, kind)[0]
+    S += np.outer(fk, v)
+    z += fk
+    den = fq @ z
+    return (fq @ S) / den if den != 0.0 else np.zeros(v.shape[0])
+
+
 # ---------------------------------------------------------------- [B, H, L, d] wrappers
 def _per_head(fn, Q, K, V, Om, *args, **kw):
     B, H = Q.shape[:2]

@@ -70,6 +70,24 @@ def _softmax_mask_slip(q, k, v, causal, rows=None):
     return (a @ v) / a.sum(axis=1, keepdims=True)
 
 
+def _decode_read_before_add(S, z, q, k, v, Om, kind):
+    fk = O.phi(k[None, :], Om, kind)[0]
+    fq = O.phi(q[None, :], Om, kind)[0]
+    den = fq @ z
+    out = (fq @ S) / den if den != 0.0 else np.zeros(v.shape[0])
+    S += np.outer(fk, v)
+    z += fk
+    return out
+
+
+def _decode_value_for_key(S, z, q, k, v, Om, kind):
+    fk = O.phi(k[None, :], Om, kind)[0]
+    fq = O.phi(q[None, :], Om, kind)[0]
+    S += np.outer(fk, k)
+    z += fk
+    return (fq @ S) / (fq @ z)
+
+
 CASES = [
     ("phi_trig", _phi_trig_no_exp, [P.test_trig_self_inner_product_identity]),
     ("phi_trig", _phi_trig_cos_twice, [P.test_trig_self_inner_product_identity]),
@@ -81,6 +99,10 @@ CASES = [
     ("gram_schmidt_rows", _gs_no_normalise, [P.test_gram_schmidt_matches_qr_with_positive_diagonal]),
     ("orf_matrix", _orf_no_chi, [lambda: P.test_orf_structure(32, 16)]),
     ("softmax_attention_head", _softmax_mask_slip, [lambda: P.test_softmax_matches_torch(True)]),
+    ("favor_decode_step_head", _decode_read_before_add,
+     [lambda: P.test_decode_steps_equal_masked_rows(O.TRIG)]),
+    ("favor_decode_step_head", _decode_value_for_key,
+     [lambda: P.test_decode_steps_equal_masked_rows(O.RELU)]),
 ]
 
 

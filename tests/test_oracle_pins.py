@@ -134,6 +134,42 @@ def test_causal_prefix_equals_masked(kind):
     np.testing.assert_allclose(cau[-1], O.favor_bidirectional_head(q, k, v, om, kind)[-1], rtol=1e-10)
 
 
+# ------------------------------------------------------------------ decode step (carried state)
+@pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
+def test_decode_steps_equal_masked_rows(kind):
+    # calls from an empty state reproduce the quadratic masked form row by row
+    L, d, M = 150, 16, 32
+    q, k, v = _qkv(L, d, seed=2)
+    om = _orf(M, d, seed=2)[0]
+    S, z = O.favor_decode_state(M, d, kind)
+    rows = np.stack([O.favor_decode_step_head(S, z, q[i], k[i], v[i], om, kind) for i in range(L)])
+    np.testing.assert_allclose(rows, O.favor_explicit_head(q, k, v, om, kind, causal=True),
+                               rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(rows[0], v[0], rtol=1e-12)
+    # the final state, read by fresh queries, is bidirectional attention over all L keys
+    qn = np.random.default_rng(5).standard_normal((7, d)) * 0.3
+    fq = O.phi(qn, om, kind)
+    np.testing.assert_allclose((fq @ S) / (fq @ z)[:, None],
+                               O.favor_explicit_head(qn, k, v, om, kind, causal=False),
+                               rtol=1e-9, atol=1e-12)
+
+
+def test_decode_state_is_order_free():
+    # the state is a sum over tokens: feeding them in another order gives the same state
+    L, d, M = 40, 8, 16
+    q, k, v = _qkv(L, d, seed=3)
+    om = _orf(M, d, seed=3)[0]
+    S1, z1 = O.favor_decode_state(M, d, O.TRIG)
+    S2, z2 = O.favor_decode_state(M, d, O.TRIG)
+    for i in range(L):
+        O.favor_decode_step_head(S1, z1, q[i], k[i], v[i], om, O.TRIG)
+    for i in np.random.default_rng(0).permutation(L):
+        O.favor_decode_step_head(S2, z2, q[i], k[i], v[i], om, O.TRIG)
+    np.testing.assert_allclose(S1, S2, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(z1, z2, rtol=1e-12, atol=1e-12)
+    assert S1.shape == (2 * M, d) and z1.shape == (2 * M,)
+
+
 # ------------------------------------------------------------------ invariants
 @pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
 @pytest.mark.parametrize("causal", [False, True])
