@@ -252,6 +252,71 @@ def run_lsweep(args):
         del sets
 
 
+def decode_bytes_per_call(B, H, d, M, kind):
+    """Algorithmic HBM bytes of one decode call: the fp32 state read and written once, q, k, v
+    read and out written (bf16), the reference read and written, Omega read once per head."""
+    F = 2 * M if kind == 0 else M
+    BH = B * H
+    return BH * (2 * F * (d + 1) * 4 + 4 * d * 2 + 8) + H * M * d * 2
+
+
+def run_decode(args):
+    """Causal decode: one token per head per call against the carried fp32 state. Two batch
+    sizes per feature map: B=512, H=8 (4096 heads; the state, 272-545 MB, is larger than twice
+    the L2, so each call streams it from HBM) and B=4, H=8 (32 heads; the 4.3 MB state stays in
+    L2: a latency point). T=64 distinct tokens are captured in one CUDA graph and replayed."""
+    import torch
+
+    import favor_inputs as fi
+    import linear_kernelized_attention_b200 as F
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    H, d, M, T = 8, 64, 256, 64
+    G, R = fi.orf_gaussians(H, M, d, seed=0)
+    omega = F.favor_orf_omega(torch.from_numpy(G).to(dev), torch.from_numpy(R).to(dev), M, dtype=torch.bfloat16)
+    for B in (512, 4):
+        q, k, v = fi.qkv(B, H, T, d, seed=7)
+        q, k, v = (fi.round_to(x, "bf16").permute(2, 0, 1, 3).contiguous().to(dev) for x in (q, k, v))
+        out = torch.empty_like(q)
+        for kind in (0, 1):
+            st = F.favor_decode_new_state(B, H, d, M, kind, device=dev, stream=stream)
+            for t in range(max(args.warmup, 3)):
+                F.favor_decode_step(q[t % T], k[t % T], v[t % T], omega, st, out=out[t % T], feature_kind=kind,
+                                    stream=stream)
+            torch.cuda.synchronize()
+            if F.favor_sync_status(stream) != 0:
+                raise RuntimeError("device status not OK")
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for t in range(T):
+                    F.favor_decode_step(q[t], k[t], v[t], omega, st, out=out[t], feature_kind=kind, stream=stream)
+            g.replay()
+            torch.cuda.synchronize()
+            reps = 10
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            if F.favor_sync_status(stream) != 0:
+                raise RuntimeError("device status not OK")
+            us = 1e3 * a.elapsed_time(b) / (reps * T)
+            nb = decode_bytes_per_call(B, H, d, M, kind)
+            gbs = nb / (us * 1e-6) / 1e9
+            print(json.dumps({
+                "decode": True, "variant": "trig" if kind == 0 else "relu", "B": B, "H": H, "d": d, "M": M,
+                "us_per_call": us, "tokens_per_s": B * H / (us * 1e-6),
+                "state_mb": F.favor_decode_state_bytes(B, H, d, M, kind) / 1e6,
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                             "bytes_per_call": nb, "peak_source": f"{peak_src} copy"}}), flush=True)
+            del g, st
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -261,9 +326,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--lsweep", action="store_true",
                     help="throughput against L (B=1, H=16, trig) instead of the bench line")
+    ap.add_argument("--decode", action="store_true",
+                    help="causal decode calls (carried state) instead of the bench line")
     args = ap.parse_args()
     if args.lsweep:
         return run_lsweep(args)
+    if args.decode:
+        return run_decode(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -159,6 +159,36 @@ int favor_attention_f32_noalloc(const float* q, const float* k, const float* v, 
 /* Size in bytes of the static workspace of favor_attention_f32_noalloc. */
 size_t favor_noalloc_scratch_bytes(void);
 
+/*
+ * Causal decode: one token per (batch, head) per call, against a carried state.
+ * The explainer's 核心机制 section: the causal prefix sums S_t = S_{t-1} + phi(k_t) v_t^T and
+ * z_t = z_{t-1} + phi(k_t), read by the same token's query: out_t = phi(q_t) S_t / phi(q_t) z_t.
+ * From a state set by favor_decode_init, calls on tokens 0 .. t return causal rows 0 .. t of
+ * favor_attention(causal = 1) on the same sequence. Each call streams the state once (an
+ * HBM-bound matrix-vector product on CUDA cores); the cost per token does not grow with t.
+ *
+ * State (owned by the caller, device memory, 16-byte aligned, favor_decode_state_bytes() bytes),
+ * fp32, three regions one after another, heads numbered bh = b*H + h:
+ *   S [B*H, F, d]   the state rows; F = 2M (trig: M cos rows, then M sin rows) or M (ReLU)
+ *   z [B*H, F]      the normaliser column
+ *   c [B*H]         the stabiliser reference: -inf when empty, then the running max of |k|^2/2
+ * Trig rows are stored as the sum of exp(|k_j|^2/2 - c) [cos(Omega k_j), sin(Omega k_j)] [v_j | 1];
+ * ReLU rows as the sum of max(Omega k_j, 0) [v_j | 1]; the factor 1/sqrt(M) is dropped (it
+ * cancels). Where c grows, S and z are rescaled by exp(c_old - c_new) in the same pass.
+ *
+ * favor_decode_step: q, k, v, out [B, H, d] bf16 (this token of every head); omega [H, M, d] bf16.
+ * Device pointers, 16-byte aligned. Reads and rewrites `state` in place; calls on one state must
+ * be ordered (one stream, or events). Arithmetic: projections, features (sincosf, expf) and the
+ * state in fp32; the row is divided in fp32 and rounded once to bf16. A zero denominator gives a
+ * zero row. Supported: d in {16, 32, 64, 128}; 1 <= M <= 512 (trig) or <= 1024 (ReLU);
+ * B*H*8 <= INT_MAX. Other shapes return FAVOR_ERR_UNSUPPORTED (or FAVOR_ERR_SHAPE for sizes
+ * that are non-positive or too large) and launch nothing.
+ */
+size_t favor_decode_state_bytes(int B, int H, int d, int M, int feature_kind); /* 0: unsupported */
+int favor_decode_init(void* state, int B, int H, int d, int M, int feature_kind, void* stream);
+int favor_decode_step(const void* q, const void* k, const void* v, const void* omega, void* state,
+                      void* out, int B, int H, int d, int M, int feature_kind, void* stream);
+
 /* Synchronise `stream`, then read and clear the device status word (FAVOR_OK or a code). */
 int favor_sync_status(void* stream);
 

@@ -7,7 +7,8 @@ if the library is missing or a call fails, an exception is raised.
 Entry points mirror the C ABI in include/favor.h:
     favor_attention, favor_attention_chunked, favor_attention_f32, favor_orf_omega,
     favor_attention_host, favor_sync_status, favor_status_string, favor_workspace_bytes,
-    favor_selftest_timeout, favor_attention_f32_noalloc, favor_noalloc_scratch_bytes
+    favor_selftest_timeout, favor_attention_f32_noalloc, favor_noalloc_scratch_bytes,
+    favor_decode_state_bytes, favor_decode_init, favor_decode_step
 """
 from __future__ import annotations
 
@@ -36,6 +37,9 @@ _SIGS = {
     "favor_workspace_bytes": (_sz, [_i] * 7),
     "favor_attention_f32_noalloc": (_i, [_vp] * 5 + [_i] * 7 + [_vp]),
     "favor_noalloc_scratch_bytes": (_sz, []),
+    "favor_decode_state_bytes": (_sz, [_i] * 5),
+    "favor_decode_init": (_i, [_vp] + [_i] * 5 + [_vp]),
+    "favor_decode_step": (_i, [_vp] * 6 + [_i] * 5 + [_vp]),
 }
 _LIB = None
 
@@ -194,3 +198,62 @@ def favor_attention_f32_noalloc(q, k, v, omega, out=None, feature_kind=FAVOR_TRI
 
 def favor_noalloc_scratch_bytes() -> int:
     return lib().favor_noalloc_scratch_bytes()
+
+
+# ---------------------------------------------------------------- causal decode (carried state)
+def favor_decode_state_bytes(B, H, d, M, feature_kind=FAVOR_TRIG) -> int:
+    return lib().favor_decode_state_bytes(B, H, d, M, int(feature_kind))
+
+
+def favor_decode_init(state, B, H, d, M, feature_kind=FAVOR_TRIG, stream=None):
+    """Set `state` (a CUDA tensor of favor_decode_state_bytes bytes) to the empty state."""
+    rc = lib().favor_decode_init(state.data_ptr(), B, H, d, M, int(feature_kind), _stream(stream))
+    _check(rc, "favor_decode_init")
+    return state
+
+
+def favor_decode_new_state(B, H, d, M, feature_kind=FAVOR_TRIG, device="cuda", stream=None):
+    """Allocate (with torch) and initialise an empty decode state: a flat float32 tensor."""
+    import torch
+    n = favor_decode_state_bytes(B, H, d, M, feature_kind)
+    if n == 0:
+        raise FavorError(-5, "favor_decode_state_bytes")
+    state = torch.empty(n // 4, dtype=torch.float32, device=device)
+    return favor_decode_init(state, B, H, d, M, feature_kind, stream)
+
+
+def favor_decode_state_views(state, B, H, d, M, feature_kind=FAVOR_TRIG):
+    """Views (S [B*H, F, d], z [B*H, F], c [B*H]) of a decode state, per include/favor.h."""
+    F = 2 * M if feature_kind == FAVOR_TRIG else M
+    BH = B * H
+    S = state[:BH * F * d].view(BH, F, d)
+    z = state[BH * F * d:BH * F * (d + 1)].view(BH, F)
+    c = state[BH * F * (d + 1):BH * F * (d + 1) + BH]
+    return S, z, c
+
+
+def favor_decode_step(q, k, v, omega, state, out=None, feature_kind=FAVOR_TRIG, stream=None):
+    """One causal decode step. q, k, v: [B, H, d] bf16 (one token per head); omega: [H, M, d]
+    bf16; state: from favor_decode_new_state, updated in place. Returns out [B, H, d] bf16."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v), ("omega", omega)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be a bfloat16 CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share the shape [B, H, d]")
+    B, H, d = q.shape
+    if omega.dim() != 3 or omega.shape[0] != H or omega.shape[2] != d:
+        raise ValueError("omega must have shape [H, M, d]")
+    M = omega.shape[1]
+    need = favor_decode_state_bytes(B, H, d, M, feature_kind)
+    if not state.is_cuda or state.numel() * state.element_size() < need:
+        raise ValueError(f"state must be a CUDA tensor of at least {need} bytes")
+    if out is None:
+        out = torch.empty_like(q)
+    rc = lib().favor_decode_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), omega.data_ptr(),
+                                 state.data_ptr(), out.data_ptr(), B, H, d, M, int(feature_kind),
+                                 _stream(stream))
+    _check(rc, "favor_decode_step")
+    return out

@@ -5,6 +5,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cstdint>
 #include <cstdio>
@@ -15,6 +16,7 @@
 #include "kernels_f32.cuh"
 #include "kernel_bidir.cuh"
 #include "kernel_causal.cuh"
+#include "kernel_decode.cuh"
 
 namespace favor {
 
@@ -378,6 +380,28 @@ int launch_f32_static(const float* q, const float* k, const float* v, const floa
 
 }  // namespace
 
+// ------------------------------------------------------------------ decode step
+int check_decode(const void* state, int B, int H, int d, int M, int kind) {
+  if (B <= 0 || H <= 0 || d <= 0 || M <= 0) return FAVOR_ERR_SHAPE;
+  if ((long long)B * H * dec::kMaxG > INT_MAX) return FAVOR_ERR_SHAPE;
+  if (kind != FAVOR_TRIG && kind != FAVOR_RELU) return FAVOR_ERR_KIND;
+  if (d != 16 && d != 32 && d != 64 && d != 128) return FAVOR_ERR_UNSUPPORTED;
+  if (M > (kind == FAVOR_TRIG ? dec::kMaxRows / 2 : dec::kMaxRows)) return FAVOR_ERR_UNSUPPORTED;
+  (void)state;
+  return FAVOR_OK;
+}
+
+long long decode_rows(int M, int kind) { return kind == FAVOR_TRIG ? 2ll * M : M; }
+
+// Cluster size: double G (<= 8) while B*H*G CTAs fill at most half the SMs and every CTA
+// keeps at least 16 angles. Large batches take G = 1 (no cluster exchange); a few heads
+// (B*H = 32) take G = 4.
+int decode_cluster(long long BH, int M) {
+  int G = 1;
+  while (G < dec::kMaxG && BH * G * 2 <= sm_count() && (M + 2 * G - 1) / (2 * G) >= 16) G *= 2;
+  return G;
+}
+
 // ====================================================================== C ABI
 extern "C" {
 
@@ -513,6 +537,72 @@ int favor_attention_f32_noalloc(const float* q, const float* k, const float* v, 
 }
 
 size_t favor_noalloc_scratch_bytes(void) { return favor::kNoAllocScratchBytes; }
+
+size_t favor_decode_state_bytes(int B, int H, int d, int M, int feature_kind) {
+  if (check_decode(nullptr, B, H, d, M, feature_kind) != FAVOR_OK) return 0;
+  const long long BH = (long long)B * H;
+  return (size_t)(BH * decode_rows(M, feature_kind) * (d + 1) + BH) * sizeof(float);
+}
+
+int favor_decode_init(void* state, int B, int H, int d, int M, int feature_kind, void* stream) {
+  if (!state) return FAVOR_ERR_NULL;
+  if (!aligned16(state)) return FAVOR_ERR_ALIGN;
+  int rc = check_decode(state, B, H, d, M, feature_kind);
+  if (rc != FAVOR_OK) return rc;
+  if ((rc = check_device()) != FAVOR_OK) return rc;
+  const long long BH = (long long)B * H;
+  const long long n_sz = BH * decode_rows(M, feature_kind) * (d + 1);
+  const long long blocks = std::min<long long>((n_sz + BH + 255) / 256, 8ll * sm_count());
+  dec::k_decode_init<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<float*>(state), n_sz, BH);
+  return cudaGetLastError() == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
+}
+
+int favor_decode_step(const void* q, const void* k, const void* v, const void* omega, void* state,
+                      void* out, int B, int H, int d, int M, int feature_kind, void* stream) {
+  if (!q || !k || !v || !omega || !state || !out) return FAVOR_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(omega) || !aligned16(state) ||
+      !aligned16(out))
+    return FAVOR_ERR_ALIGN;
+  int rc = check_decode(state, B, H, d, M, feature_kind);
+  if (rc != FAVOR_OK) return rc;
+  if ((rc = check_device()) != FAVOR_OK) return rc;
+  const long long BH = (long long)B * H, F = decode_rows(M, feature_kind);
+  dec::DecodeParams prm{};
+  prm.z_off = BH * F * d;
+  prm.c_off = BH * F * (d + 1);
+  prm.BH = (int)BH;
+  prm.H = H;
+  prm.d = d;
+  prm.M = M;
+  prm.kind = feature_kind;
+  prm.G = decode_cluster(BH, M);
+  prm.na = (M + prm.G - 1) / prm.G;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(BH * prm.G));
+  cfg.blockDim = dim3(dec::kThreads);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = prm.G;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void (*kern)(const __nv_bfloat16*, const __nv_bfloat16*, const __nv_bfloat16*, const __nv_bfloat16*, float*,
+               __nv_bfloat16*, const dec::DecodeParams) = d == 16   ? dec::k_decode_step<16>
+                                                         : d == 32 ? dec::k_decode_step<32>
+                                                         : d == 64 ? dec::k_decode_step<64>
+                                                                   : dec::k_decode_step<128>;
+  if ((rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), dec::kSmemBytes)) != FAVOR_OK) return rc;
+  cfg.dynamicSmemBytes = dec::kSmemBytes;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(q),
+                            static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+                            static_cast<const __nv_bfloat16*>(omega), static_cast<float*>(state),
+                            static_cast<__nv_bfloat16*>(out), prm) == cudaSuccess
+             ? FAVOR_OK
+             : FAVOR_ERR_CUDA;
+}
 
 // Launch the bounded-wait self-test: a wait that nothing satisfies, limited to `limit_cycles`.
 // favor_sync_status() afterwards must report FAVOR_ERR_TIMEOUT.

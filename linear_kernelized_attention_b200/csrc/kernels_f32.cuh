@@ -9,6 +9,8 @@
 //     Causal: S_i = (prefix before the chunk) + sum_{j in chunk, j <= i} phi(k_j)[v_j|1]^T.
 // Cancelling factors: 1/sqrt(M) and exp(|q|^2/2) are dropped, and the key factor is
 // exp(|k|^2/2 - c_h) with c_h = max_j |k_j|^2/2 of the head.
+// sin, cos and exp are evaluated in double and rounded to fp32: the library is built with fast
+// single-precision intrinsics, whose error grows with the angle.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -33,9 +35,9 @@ __device__ __forceinline__ float feature_value(int kind, int M, int f, const flo
   float u = 0.f;
   for (int t = 0; t < d; ++t) u = fmaf(om[t], x[t], u);
   if (kind == 0) {
-    float s, c;
-    sincosf(u, &s, &c);
-    return w * (f < M ? c : s);
+    double s, c;
+    sincos(static_cast<double>(u), &s, &c);
+    return w * static_cast<float>(f < M ? c : s);
   }
   return fmaxf(u, 0.f);
 }
@@ -92,7 +94,7 @@ __global__ void __launch_bounds__(kThreads)
       if (kind == 0) {
         float s = 0.f;
         for (int t = 0; t < d; ++t) s = fmaf(sk[j * d + t], sk[j * d + t], s);
-        w = expf(0.5f * s - cmax[bh]);
+        w = static_cast<float>(exp(0.5 * static_cast<double>(s) - cmax[bh]));
       } else {
         w = 1.f;
       }
@@ -171,7 +173,7 @@ __global__ void __launch_bounds__(kThreads)
       if (kind == 0) {
         float s = 0.f;
         for (int t = 0; t < d; ++t) s = fmaf(sk[j * d + t], sk[j * d + t], s);
-        w = expf(0.5f * s - cmax[bh]);
+        w = static_cast<float>(exp(0.5 * static_cast<double>(s) - cmax[bh]));
       } else {
         w = 1.f;
       }

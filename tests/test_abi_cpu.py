@@ -74,3 +74,44 @@ def test_f32_and_orf_validation():
 def test_workspace_bytes_is_host_only():
     assert F.favor_workspace_bytes(1, 1, 1, 64, 64, 0, False) >= 0
     assert F.favor_workspace_bytes(0, 1, 1, 64, 64, 0, False) == 0
+
+
+# ------------------------------------------------------------------ decode entry points
+@pytest.mark.parametrize("B,H,d,M,kind", [(1, 1, 64, 256, 0), (4, 8, 64, 256, 1), (2, 3, 128, 512, 0),
+                                          (1, 2, 16, 1024, 1)])
+def test_decode_state_bytes(B, H, d, M, kind):
+    F_ = 2 * M if kind == 0 else M
+    assert F.favor_decode_state_bytes(B, H, d, M, kind) == 4 * (B * H * F_ * (d + 1) + B * H)
+
+
+@pytest.mark.parametrize("args", [(1, 1, 48, 64, 0), (1, 1, 64, 513, 0), (1, 1, 64, 1025, 1),
+                                  (0, 1, 64, 64, 0), (1, 1, 64, 64, 2)])
+def test_decode_state_bytes_unsupported_is_zero(args):
+    assert F.favor_decode_state_bytes(*args) == 0
+
+
+def _dec(**over):
+    a = dict(q=16, k=32, v=48, om=64, st=80, out=96, B=1, H=1, d=64, M=64, kind=0)
+    a.update(over)
+    vp = ctypes.c_void_p
+    return F.lib().favor_decode_step(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["om"]), vp(a["st"]),
+                                     vp(a["out"]), a["B"], a["H"], a["d"], a["M"], a["kind"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    ({"q": 0}, -1), ({"st": 0}, -1), ({"out": 0}, -1),
+    ({"v": 50}, -2), ({"st": 84}, -2),
+    ({"B": 0}, -3), ({"M": -4}, -3), ({"H": 1 << 30}, -3),
+    ({"kind": 3}, -4),
+    ({"d": 48}, -5), ({"d": 256}, -5), ({"M": 513}, -5), ({"M": 1025, "kind": 1}, -5),
+])
+def test_decode_validation_rejects_before_any_cuda_call(over, code):
+    assert _dec(**over) == code
+
+
+def test_decode_init_validation():
+    vp = ctypes.c_void_p
+    assert F.lib().favor_decode_init(vp(0), 1, 1, 64, 64, 0, None) == -1
+    assert F.lib().favor_decode_init(vp(20), 1, 1, 64, 64, 0, None) == -2
+    assert F.lib().favor_decode_init(vp(32), 1, 1, 64, 64, 5, None) == -4
+    assert F.lib().favor_decode_init(vp(32), 1, 1, 40, 64, 0, None) == -5
