@@ -278,11 +278,13 @@ def run_decode(args):
     H, d, M, T = 8, 64, 256, 64
     G, R = fi.orf_gaussians(H, M, d, seed=0)
     omega = F.favor_orf_omega(torch.from_numpy(G).to(dev), torch.from_numpy(R).to(dev), M, dtype=torch.bfloat16)
-    for B in (512, 4):
+    batches = [int(x) for x in args.decode_batches.split(",")]
+    kinds = [{"trig": 0, "relu": 1}[x] for x in args.decode_kinds.split(",")]
+    for B in batches:
         q, k, v = fi.qkv(B, H, T, d, seed=7)
         q, k, v = (fi.round_to(x, "bf16").permute(2, 0, 1, 3).contiguous().to(dev) for x in (q, k, v))
         out = torch.empty_like(q)
-        for kind in (0, 1):
+        for kind in kinds:
             st = F.favor_decode_new_state(B, H, d, M, kind, device=dev, stream=stream)
             for t in range(max(args.warmup, 3)):
                 F.favor_decode_step(q[t % T], k[t % T], v[t % T], omega, st, out=out[t % T], feature_kind=kind,
@@ -328,6 +330,8 @@ def main():
                     help="throughput against L (B=1, H=16, trig) instead of the bench line")
     ap.add_argument("--decode", action="store_true",
                     help="causal decode calls (carried state) instead of the bench line")
+    ap.add_argument("--decode-batches", default="512,4", help="batch sizes B for --decode (H=8)")
+    ap.add_argument("--decode-kinds", default="trig,relu", help="feature maps for --decode")
     args = ap.parse_args()
     if args.lsweep:
         return run_lsweep(args)

@@ -283,8 +283,12 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode_step(const __nv_bfloat16
     }
     part[n] = t;
   }
-  // Every CTA's partial is in its shared memory; rank 0 sums them.
-  cluster_sync();
+  // Every CTA's partial is in its shared memory; rank 0 sums them. A cluster barrier (its release
+  // waits for this CTA's HBM stores) is taken only when there is another CTA to read from.
+  if (G > 1)
+    cluster_sync();
+  else
+    __syncthreads();
   if (rank == 0) {
     if (tid <= d4) {
       float4 t = reinterpret_cast<const float4*>(part)[tid];
@@ -306,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode_step(const __nv_bfloat16
     if (tid == 0 && trig) *cref = sc[2];  // every CTA of the cluster read c before the barrier
   }
   // The other CTAs keep their shared memory until rank 0 has read it.
-  cluster_sync();
+  if (G > 1) cluster_sync();
 }
 
 // Empty state: S = 0, z = 0 and every reference -inf.
