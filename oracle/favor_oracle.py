@@ -81,6 +81,65 @@ def orf_matrices(G: np.ndarray, R: np.ndarray, M: int) -> np.ndarray:
     return np.stack([orf_matrix(G[h], R[h], M) for h in range(G.shape[0])])
 
 
+# ---------------------------------------------------------------- counter-based draws
+# The ORF directions and lengths are Gaussian draws ([EXPL, 核心机制]; [MLMP-zh, 方法详解]).
+# To redraw Omega on the device from a seed, both sides generate the draws with the same
+# counter-based generator, each from its published definition: Philox4x64 with 10 rounds
+# (Salmon, Moraes, Dror and Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3", SC 2011).
+_M64 = (1 << 64) - 1
+PHILOX_M0, PHILOX_M1 = 0xD2E7470EE14C6C93, 0xCA5A826395121157   # round multipliers
+PHILOX_W0, PHILOX_W1 = 0x9E3779B97F4A7C15, 0xBB67AE8584CAA73B   # key increments (Weyl)
+
+
+def philox4x64_10(counter, key):
+    """One Philox4x64-10 block: counter (4 words) and key (2 words) -> 4 uint64 words.
+
+    Python integers, so every product and xor is exact. A round maps
+    (x0, x1, x2, x3) to (hi(M1 x2) ^ x1 ^ k0, lo(M1 x2), hi(M0 x0) ^ x3 ^ k1, lo(M0 x0));
+    the key gains (W0, W1) between rounds.
+    """
+    x0, x1, x2, x3 = (int(c) & _M64 for c in counter)
+    k0, k1 = (int(k) & _M64 for k in key)
+    for r in range(10):
+        if r:
+            k0, k1 = (k0 + PHILOX_W0) & _M64, (k1 + PHILOX_W1) & _M64
+        p0, p1 = PHILOX_M0 * x0, PHILOX_M1 * x2
+        x0, x1, x2, x3 = ((p1 >> 64) ^ x1 ^ k0, p1 & _M64, (p0 >> 64) ^ x3 ^ k1, p0 & _M64)
+    return [x0, x1, x2, x3]
+
+
+def philox_normals(seed, group):
+    """Four N(0, 1) draws of group `group`: Philox4x64-10 of counter (group, 0, 0, 0) and key
+    (seed, 0); each word w gives u = (floor(w / 2^11) + 1/2) 2^-53 in (0, 1), and the pairs
+    (u0, u1), (u2, u3) go through Box-Muller: sqrt(-2 ln u_a) (cos, sin)(2 pi u_b)."""
+    w = philox4x64_10([group, 0, 0, 0], [seed, 0])
+    u = [((x >> 11) + 0.5) * 2.0 ** -53 for x in w]
+    out = []
+    for a, b in ((u[0], u[1]), (u[2], u[3])):
+        r, t = np.sqrt(-2.0 * np.log(a)), 2.0 * np.pi * b
+        out += [r * np.cos(t), r * np.sin(t)]
+    return out
+
+
+def seeded_orf_gaussians(seed, H, M, d):
+    """The ORF draws of seed `seed`: G [H, ceil(M/d), d, d] and R [H, M, d].
+
+    Draw n of the stream is normal n % 4 of group n // 4. G[h, b, i, j] is draw
+    ((h nb + b) d + i) d + j; R[h, r, j] is draw NG + (h M + r) d + j, with NG the size of G
+    rounded up to a multiple of 4.
+    """
+    nb = -(-M // d)
+    ng = H * nb * d * d
+    NG = -(-ng // 4) * 4
+    total = NG + H * M * d
+    draws = np.empty(-(-total // 4) * 4)
+    for g in range(len(draws) // 4):
+        draws[4 * g:4 * g + 4] = philox_normals(seed, g)
+    G = draws[:ng].reshape(H, nb, d, d)
+    R = draws[NG:NG + H * M * d].reshape(H, M, d)
+    return G, R
+
+
 # ---------------------------------------------------------------- feature maps
 def phi_trig(X: np.ndarray, Om: np.ndarray) -> np.ndarray:
     """Trigonometric softmax-kernel features [L, 2M] of the rows of X [L, d].

@@ -88,6 +88,28 @@ def _decode_value_for_key(S, z, q, k, v, Om, kind):
     return (fq @ S) / (fq @ z)
 
 
+def _philox_wrong_weyl(counter, key):
+    M64 = (1 << 64) - 1
+    x0, x1, x2, x3 = (int(c) & M64 for c in counter)
+    k0, k1 = (int(k) & M64 for k in key)
+    for r in range(10):
+        if r:
+            k0, k1 = (k0 + O.PHILOX_W1) & M64, (k1 + O.PHILOX_W0) & M64
+        p0, p1 = O.PHILOX_M0 * x0, O.PHILOX_M1 * x2
+        x0, x1, x2, x3 = ((p1 >> 64) ^ x1 ^ k0, p1 & M64, (p0 >> 64) ^ x3 ^ k1, p0 & M64)
+    return [x0, x1, x2, x3]
+
+
+def _normals_cos_twice(seed, group):
+    w = O.philox4x64_10([group, 0, 0, 0], [seed, 0])
+    u = [((x >> 11) + 0.5) * 2.0 ** -53 for x in w]
+    out = []
+    for a, b in ((u[0], u[1]), (u[2], u[3])):
+        r, t = np.sqrt(-2.0 * np.log(a)), 2.0 * np.pi * b
+        out += [r * np.cos(t), r * np.cos(t)]
+    return out
+
+
 CASES = [
     ("phi_trig", _phi_trig_no_exp, [P.test_trig_self_inner_product_identity]),
     ("phi_trig", _phi_trig_cos_twice, [P.test_trig_self_inner_product_identity]),
@@ -99,6 +121,8 @@ CASES = [
     ("gram_schmidt_rows", _gs_no_normalise, [P.test_gram_schmidt_matches_qr_with_positive_diagonal]),
     ("orf_matrix", _orf_no_chi, [lambda: P.test_orf_structure(32, 16)]),
     ("softmax_attention_head", _softmax_mask_slip, [lambda: P.test_softmax_matches_torch(True)]),
+    ("philox4x64_10", _philox_wrong_weyl, [lambda: P.test_philox_matches_numpy_bit_generator(5, 0)]),
+    ("philox_normals", _normals_cos_twice, [P.test_philox_normals_box_muller_form]),
     ("favor_decode_step_head", _decode_read_before_add,
      [lambda: P.test_decode_steps_equal_masked_rows(O.TRIG)]),
     ("favor_decode_step_head", _decode_value_for_key,

@@ -170,6 +170,63 @@ def test_decode_state_is_order_free():
     assert S1.shape == (2 * M, d) and z1.shape == (2 * M,)
 
 
+# ------------------------------------------------------------------ counter-based ORF draws
+def _words(x, n):
+    return [(x >> (64 * i)) & ((1 << 64) - 1) for i in range(n)]
+
+
+@pytest.mark.parametrize("key,counter", [(0, 0), (5, 0), (2**64 + 3, 2**64 - 3), (2**128 - 1, 2**200 + 2**64 - 2),
+                                         (0x243F6A8885A308D3, 0x13198A2E03707344)])
+def test_philox_matches_numpy_bit_generator(key, counter):
+    # numpy's Philox bit generator (its own C implementation) advances the counter before each
+    # block: its outputs 4i .. 4i+3 are the block of counter + 1 + i
+    raw = np.random.Philox(key=key, counter=counter).random_raw(24)
+    mine = []
+    for i in range(6):
+        mine += O.philox4x64_10(_words((counter + 1 + i) % 2**256, 4), _words(key, 2))
+    assert [int(x) for x in raw] == mine
+
+
+def test_philox_normals_are_standard_normal():
+    from scipy import stats
+    z = np.array([x for g in range(5000) for x in O.philox_normals(11, g)])
+    assert abs(z.mean()) < 4 / np.sqrt(z.size) and abs(z.var() - 1) < 6 * np.sqrt(2 / z.size)
+    assert stats.kstest(z, "norm").pvalue > 1e-3
+    # the two members of a Box-Muller pair are uncorrelated, and so are neighbouring groups
+    assert abs(np.corrcoef(z[0::2], z[1::2])[0, 1]) < 4 / np.sqrt(z.size / 2)
+    assert abs(np.corrcoef(z[:-4], z[4:])[0, 1]) < 4 / np.sqrt(z.size)
+
+
+def test_philox_normals_box_muller_form():
+    # the words map to u in (0, 1) and a pair (u_a, u_b) to sqrt(-2 ln u_a) (cos, sin)(2 pi u_b):
+    # the squared norm of each pair is -2 ln u_a, whatever u_b
+    for g in (0, 7, 123456789):
+        w = O.philox4x64_10([g, 0, 0, 0], [3, 0])
+        z = O.philox_normals(3, g)
+        for p in range(2):
+            ua = ((w[2 * p] >> 11) + 0.5) * 2.0 ** -53
+            assert 0.0 < ua < 1.0
+            assert z[2 * p] ** 2 + z[2 * p + 1] ** 2 == pytest.approx(-2.0 * math.log(ua), rel=1e-13)
+
+
+def test_seeded_orf_gaussians_layout():
+    H, M, d, seed = 2, 40, 8, 9
+    G, R = O.seeded_orf_gaussians(seed, H, M, d)
+    nb = 5
+    assert G.shape == (H, nb, d, d) and R.shape == (H, M, d)
+    NG = -(-H * nb * d * d // 4) * 4
+    for (h, b, i, j) in [(0, 0, 0, 0), (1, 4, 7, 7), (1, 2, 3, 5)]:
+        n = ((h * nb + b) * d + i) * d + j
+        assert G[h, b, i, j] == O.philox_normals(seed, n // 4)[n % 4]
+    for (h, r, j) in [(0, 0, 0), (1, 39, 7), (0, 17, 2)]:
+        n = NG + (h * M + r) * d + j
+        assert R[h, r, j] == O.philox_normals(seed, n // 4)[n % 4]
+    # a different seed gives different draws; the same seed the same draws
+    G2, _ = O.seeded_orf_gaussians(seed + 1, H, M, d)
+    assert not np.allclose(G, G2)
+    assert np.array_equal(G, O.seeded_orf_gaussians(seed, H, M, d)[0])
+
+
 # ------------------------------------------------------------------ invariants
 @pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
 @pytest.mark.parametrize("causal", [False, True])
