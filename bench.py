@@ -319,6 +319,36 @@ def run_decode(args):
             del g, st
 
 
+def run_orf(args):
+    """Omega redrawn on the device from a seed (favor_orf_omega_seeded), bf16 output: microseconds
+    per call at H = 8 and H = 64 heads, M = 256, d = 64, each call a new seed."""
+    import torch
+
+    import linear_kernelized_attention_b200 as F
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    for H in (8, 64):
+        M, d = 256, 64
+        om = torch.empty((H, M, d), dtype=torch.bfloat16, device=dev)
+        for s in range(max(args.warmup, 3)):
+            F.favor_orf_omega_seeded(s, H, M, d, out=om, stream=stream)
+        torch.cuda.synchronize()
+        n = 50
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for s in range(n):
+            F.favor_orf_omega_seeded(1000 + s, H, M, d, out=om, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if F.favor_sync_status(stream) != 0:
+            raise RuntimeError("device status not OK")
+        us = 1e3 * a.elapsed_time(b) / n
+        print(json.dumps({"orf": True, "H": H, "M": M, "d": d, "us_per_call": us,
+                          "blocks": H * (-(-M // d)), "dtype": "bf16 out, fp64 Gram-Schmidt"}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -332,7 +362,10 @@ def main():
                     help="causal decode calls (carried state) instead of the bench line")
     ap.add_argument("--decode-batches", default="512,4", help="batch sizes B for --decode (H=8)")
     ap.add_argument("--decode-kinds", default="trig,relu", help="feature maps for --decode")
+    ap.add_argument("--orf", action="store_true", help="time Omega redrawn on the device from a seed")
     args = ap.parse_args()
+    if args.orf:
+        return run_orf(args)
     if args.lsweep:
         return run_lsweep(args)
     if args.decode:

@@ -125,6 +125,39 @@ int favor_orf_omega(const double* gauss_blocks, const double* gauss_norms, void*
                     int H, int M, int d, int omega_dtype, void* stream);
 
 /*
+ * ORF Omega redrawn on the device from a seed: as favor_orf_omega, with the Gaussian draws
+ * generated in the kernel instead of read from memory (no scratch). A new seed per call gives a
+ * new draw of the orthogonal random features (the pages' ORF: "Masked Language Modeling for
+ * Proteins via Linearly Scalable Long-Context Transformers", 方法详解 and 实验设计; the explainer's
+ * 核心机制 section).
+ * The draws: Philox4x64 with 10 rounds (Salmon, Moraes, Dror and Shaw, SC 2011), counter
+ * (g, 0, 0, 0) and key (seed, 0) for group g. Each 64-bit word w gives
+ * u = (floor(w / 2^11) + 1/2) 2^-53, and Box-Muller turns (u0, u1) and (u2, u3) into
+ * sqrt(-2 ln u_a) (cos, sin)(2 pi u_b) in double. Draw n is normal n % 4 of group n / 4.
+ * gauss_blocks[h, b, i, j] is draw ((h nb + b) d + i) d + j, with nb = ceil(M/d). gauss_norms[h, r, j]
+ * is draw NG + (h M + r) d + j, with NG = H nb d d rounded up to a multiple of 4. Those are
+ * exactly the arrays favor_orf_gaussians_seeded writes.
+ * omega: device output [H, M, d], 16-byte aligned, dtype per omega_dtype (0 = float, 1 = bf16).
+ * Supported: 1 <= d <= 128, 1 <= M, 1 <= H <= 65535.
+ */
+int favor_orf_omega_seeded(uint64_t seed, void* omega, int H, int M, int d, int omega_dtype, void* stream);
+
+/*
+ * The Gaussian draws behind favor_orf_omega_seeded, written out. gauss_blocks: device double
+ * [H, ceil(M/d), d, d]; gauss_norms: device double [H, M, d]; both 16-byte aligned.
+ * favor_orf_omega on these arrays gives the same Omega as favor_orf_omega_seeded(seed).
+ */
+int favor_orf_gaussians_seeded(uint64_t seed, double* gauss_blocks, double* gauss_norms, int H, int M, int d,
+                               void* stream);
+
+/*
+ * The raw generator: out[4 i + w] = word w of Philox4x64-10 applied to counter
+ * (first_counter + i, 0, 0, 0) with key (key, 0), for i < n_blocks (1 <= n_blocks <= 2^40).
+ * out is device memory, 16-byte aligned, 4 n_blocks uint64 words.
+ */
+int favor_philox4x64(uint64_t key, uint64_t first_counter, uint64_t n_blocks, uint64_t* out, void* stream);
+
+/*
  * Host-buffer convenience entry: q, k, v, omega, out are HOST pointers (pinned memory
  * makes the copies asynchronous). Allocates device buffers with cudaMallocAsync on
  * `stream`, copies in, runs favor_attention (dtype_code 1 = bf16) or favor_attention_f32

@@ -8,7 +8,8 @@ Entry points mirror the C ABI in include/favor.h:
     favor_attention, favor_attention_chunked, favor_attention_f32, favor_orf_omega,
     favor_attention_host, favor_sync_status, favor_status_string, favor_workspace_bytes,
     favor_selftest_timeout, favor_attention_f32_noalloc, favor_noalloc_scratch_bytes,
-    favor_decode_state_bytes, favor_decode_init, favor_decode_step
+    favor_decode_state_bytes, favor_decode_init, favor_decode_step, favor_orf_omega_seeded,
+    favor_orf_gaussians_seeded, favor_philox4x64
 """
 from __future__ import annotations
 
@@ -24,7 +25,7 @@ STATUS = {
 }
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfavor.so")
 
-_vp, _i, _ll, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t
+_vp, _i, _ll, _sz, _u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t, ctypes.c_uint64
 _SIGS = {
     "favor_attention": (_i, [_vp] * 5 + [_i] * 7 + [_vp]),
     "favor_attention_chunked": (_i, [_vp] * 5 + [_i] * 8 + [_vp]),
@@ -40,6 +41,9 @@ _SIGS = {
     "favor_decode_state_bytes": (_sz, [_i] * 5),
     "favor_decode_init": (_i, [_vp] + [_i] * 5 + [_vp]),
     "favor_decode_step": (_i, [_vp] * 6 + [_i] * 5 + [_vp]),
+    "favor_orf_omega_seeded": (_i, [_u64, _vp] + [_i] * 4 + [_vp]),
+    "favor_orf_gaussians_seeded": (_i, [_u64, _vp, _vp] + [_i] * 3 + [_vp]),
+    "favor_philox4x64": (_i, [_u64, _u64, _u64, _vp, _vp]),
 }
 _LIB = None
 
@@ -256,4 +260,39 @@ def favor_decode_step(q, k, v, omega, state, out=None, feature_kind=FAVOR_TRIG, 
                                  state.data_ptr(), out.data_ptr(), B, H, d, M, int(feature_kind),
                                  _stream(stream))
     _check(rc, "favor_decode_step")
+    return out
+
+
+# ---------------------------------------------------------------- ORF redrawn from a seed
+def favor_orf_omega_seeded(seed, H, M, d, dtype=None, out=None, device="cuda", stream=None):
+    """ORF Omega [H, M, d] drawn on the device from `seed` (Philox4x64-10; see include/favor.h)."""
+    import torch
+    dtype = dtype or torch.bfloat16
+    if out is None:
+        out = torch.empty((H, M, d), dtype=dtype, device=device)
+    code = {torch.float32: 0, torch.bfloat16: 1}[out.dtype]
+    rc = lib().favor_orf_omega_seeded(int(seed) & (2**64 - 1), out.data_ptr(), H, M, d, code, _stream(stream))
+    _check(rc, "favor_orf_omega_seeded")
+    return out
+
+
+def favor_orf_gaussians_seeded(seed, H, M, d, device="cuda", stream=None):
+    """The draws behind favor_orf_omega_seeded: (G [H, ceil(M/d), d, d], R [H, M, d]) float64."""
+    import torch
+    nb = -(-M // d)
+    G = torch.empty((H, nb, d, d), dtype=torch.float64, device=device)
+    R = torch.empty((H, M, d), dtype=torch.float64, device=device)
+    rc = lib().favor_orf_gaussians_seeded(int(seed) & (2**64 - 1), G.data_ptr(), R.data_ptr(), H, M, d,
+                                          _stream(stream))
+    _check(rc, "favor_orf_gaussians_seeded")
+    return G, R
+
+
+def favor_philox4x64(key, first_counter, n_blocks, device="cuda", stream=None):
+    """Raw Philox4x64-10 blocks: an int64 tensor [n_blocks, 4] holding the uint64 words' bits."""
+    import torch
+    out = torch.empty((n_blocks, 4), dtype=torch.int64, device=device)
+    rc = lib().favor_philox4x64(int(key) & (2**64 - 1), int(first_counter) & (2**64 - 1), int(n_blocks),
+                                out.data_ptr(), _stream(stream))
+    _check(rc, "favor_philox4x64")
     return out

@@ -402,6 +402,23 @@ int decode_cluster(long long BH, int M) {
   return G;
 }
 
+// ------------------------------------------------------------------ ORF
+// One CTA per (d x d block, head): Gram-Schmidt in fp64 shared memory, rows scaled by chi
+// lengths. The Gaussians come from G and R, or (seeded) from the Philox stream of `seed`.
+int launch_orf(const double* G, const double* R, void* omega, int H, int M, int d, int omega_dtype, uint64_t seed,
+               int seeded, cudaStream_t st) {
+  if (H <= 0 || M <= 0 || d <= 0) return FAVOR_ERR_SHAPE;
+  if (d > 128 || H > 65535) return FAVOR_ERR_UNSUPPORTED;
+  if (omega_dtype != 0 && omega_dtype != 1) return FAVOR_ERR_UNSUPPORTED;
+  int rc = check_device();
+  if (rc != FAVOR_OK) return rc;
+  const int nb = (M + d - 1) / d;
+  const size_t smem = (size_t)d * d * sizeof(double);
+  if ((rc = ensure_smem_attr(reinterpret_cast<const void*>(k_orf), (int)smem)) != FAVOR_OK) return rc;
+  k_orf<<<dim3(nb, H), 256, smem, st>>>(G, R, omega, H, M, d, omega_dtype, seed, seeded);
+  return cudaGetLastError() == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
+}
+
 // ====================================================================== C ABI
 extern "C" {
 
@@ -472,17 +489,41 @@ int favor_orf_omega(const double* gauss_blocks, const double* gauss_norms, void*
                     int d, int omega_dtype, void* stream) {
   if (!gauss_blocks || !gauss_norms || !omega) return FAVOR_ERR_NULL;
   if (!aligned16(gauss_blocks) || !aligned16(gauss_norms) || !aligned16(omega)) return FAVOR_ERR_ALIGN;
+  return launch_orf(gauss_blocks, gauss_norms, omega, H, M, d, omega_dtype, 0, 0,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int favor_orf_omega_seeded(uint64_t seed, void* omega, int H, int M, int d, int omega_dtype, void* stream) {
+  if (!omega) return FAVOR_ERR_NULL;
+  if (!aligned16(omega)) return FAVOR_ERR_ALIGN;
+  return launch_orf(nullptr, nullptr, omega, H, M, d, omega_dtype, seed, 1, static_cast<cudaStream_t>(stream));
+}
+
+int favor_orf_gaussians_seeded(uint64_t seed, double* gauss_blocks, double* gauss_norms, int H, int M, int d,
+                               void* stream) {
+  if (!gauss_blocks || !gauss_norms) return FAVOR_ERR_NULL;
+  if (!aligned16(gauss_blocks) || !aligned16(gauss_norms)) return FAVOR_ERR_ALIGN;
   if (H <= 0 || M <= 0 || d <= 0) return FAVOR_ERR_SHAPE;
   if (d > 128 || H > 65535) return FAVOR_ERR_UNSUPPORTED;
-  if (omega_dtype != 0 && omega_dtype != 1) return FAVOR_ERR_UNSUPPORTED;
   int rc = check_device();
   if (rc != FAVOR_OK) return rc;
-  const int nb = (M + d - 1) / d;
-  const size_t smem = (size_t)d * d * sizeof(double);
-  if (cudaFuncSetAttribute(k_orf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return FAVOR_ERR_CUDA;
-  k_orf<<<dim3(nb, H), 256, smem, static_cast<cudaStream_t>(stream)>>>(gauss_blocks, gauss_norms, omega, H,
-                                                                        M, d, omega_dtype);
+  const long long nb = (M + d - 1) / d, ng = H * nb * d * d, NG = (ng + 3) / 4 * 4, nr = (long long)H * M * d;
+  const long long groups = (NG + nr + 3) / 4;
+  const long long blocks = std::min<long long>((groups + 255) / 256, 8ll * sm_count());
+  rng::k_orf_gaussians<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(seed, gauss_blocks,
+                                                                                         gauss_norms, ng, NG, nr);
+  return cudaGetLastError() == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
+}
+
+int favor_philox4x64(uint64_t key, uint64_t first_counter, uint64_t n_blocks, uint64_t* out, void* stream) {
+  if (!out) return FAVOR_ERR_NULL;
+  if (!aligned16(out)) return FAVOR_ERR_ALIGN;
+  if (n_blocks == 0 || n_blocks > (1ull << 40)) return FAVOR_ERR_SHAPE;
+  int rc = check_device();
+  if (rc != FAVOR_OK) return rc;
+  const unsigned long long blocks = std::min<unsigned long long>((n_blocks + 255) / 256, 8ull * sm_count());
+  rng::k_philox_raw<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(key, first_counter, n_blocks,
+                                                                                      out);
   return cudaGetLastError() == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
 

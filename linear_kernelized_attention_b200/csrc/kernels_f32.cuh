@@ -15,6 +15,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "philox.cuh"
 #include "ptx.cuh"
 
 namespace favor {
@@ -255,44 +256,71 @@ __global__ void __launch_bounds__(kThreads)
 
 // ------------------------------------------------------------------ ORF builder
 // One block per (head, d x d Gaussian block). Rows are orthonormalised in order by classical
-// Gram-Schmidt applied twice (fp64), then row r is scaled by |gauss_norms[h, r, :]|.
+// Gram-Schmidt applied twice (fp64), then row r is scaled by |gauss_norms[h, r, :]|. With
+// `seeded`, the block's Gaussians and its rows' chi draws are generated here from `seed`
+// (philox.cuh: the same draws k_orf_gaussians writes out) instead of being read from G and R.
 // "Masked Language Modeling for Proteins via Linearly Scalable Long-Context Transformers"
 // (方法详解) calls these orthogonal random features. The explainer's 核心机制 section
 // constrains the directions to a random subsample of an orthogonal matrix.
 __global__ void __launch_bounds__(256)
     k_orf(const double* __restrict__ G, const double* __restrict__ R, void* __restrict__ omega,
-          int H, int M, int d, int out_bf16) {
+          int H, int M, int d, int out_bf16, uint64_t seed, int seeded) {
   extern __shared__ double sq[];  // [d][d] rows being orthonormalised
   __shared__ double dots[128];
   __shared__ double snorm;
   const int h = blockIdx.y, blk = blockIdx.x, nb = gridDim.x;
-  const double* g = G + (((size_t)h * nb + blk) * d) * d;
-  for (int i = threadIdx.x; i < d * d; i += blockDim.x) sq[i] = g[i];
+  const long long n0 = (((long long)h * nb + blk) * d) * d;  // first draw of this block
+  const long long NG = ((long long)H * nb * d * d + 3) / 4 * 4;
+  if (seeded) {
+    for (long long gq = n0 / 4 + threadIdx.x; gq <= (n0 + d * d - 1) / 4; gq += blockDim.x) {
+      double z[4];
+      rng::normals4(seed, (uint64_t)gq, z);
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const long long e = 4 * gq + p - n0;
+        if (e >= 0 && e < (long long)d * d) sq[e] = z[p];
+      }
+    }
+  } else {
+    const double* g = G + n0;
+    for (int i = threadIdx.x; i < d * d; i += blockDim.x) sq[i] = g[i];
+  }
   __syncthreads();
+  // Row i: two classical Gram-Schmidt passes against rows 0 .. i-1, then normalisation.
+  // Dot products: 8 lanes per row j (32 rows per sweep). Update of v: kTpt lanes per column t,
+  // each summing every kTpt-th j, combined by shuffles (kTpt a power of two <= 32 dividing 32).
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int tpt = 1;
+  while (tpt * 2 <= 32 && tpt * 2 * d <= (int)blockDim.x) tpt *= 2;
+  const int sub8 = threadIdx.x & 7, grp = threadIdx.x >> 3, ngrp = blockDim.x >> 3;
+  const int col = threadIdx.x / tpt, part = threadIdx.x % tpt;
   for (int i = 0; i < d; ++i) {
     double* vi = sq + (size_t)i * d;
-    for (int pass = 0; pass < 2; ++pass) {
-      if (i == 0) break;
-      // dots_j = q_j . v for j < i
-      for (int j = threadIdx.x; j < i; j += blockDim.x) {
-        const double* qj = sq + (size_t)j * d;
+    for (int pass = 0; pass < 2 && i > 0; ++pass) {
+      for (int j0 = 0; j0 < i; j0 += ngrp) {  // uniform trip count across the block
+        const int j = j0 + grp;
         double s = 0.0;
-        for (int t = 0; t < d; ++t) s = fma(qj[t], vi[t], s);
-        dots[j] = s;
+        if (j < i)
+          for (int t = sub8; t < d; t += 8) s = fma(sq[(size_t)j * d + t], vi[t], s);
+        s += __shfl_xor_sync(0xffffffffu, s, 4);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        if (sub8 == 0 && j < i) dots[j] = s;
       }
       __syncthreads();
-      // v -= sum_j dots_j q_j
-      for (int t = threadIdx.x; t < d; t += blockDim.x) {
-        double s = 0.0;
-        for (int j = 0; j < i; ++j) s = fma(dots[j], sq[(size_t)j * d + t], s);
-        vi[t] -= s;
-      }
+      double s = 0.0;
+      if (col < d)
+        for (int j = part; j < i; j += tpt) s = fma(dots[j], sq[(size_t)j * d + col], s);
+      for (int o = tpt >> 1; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (col < d && part == 0) vi[col] -= s;
       __syncthreads();
     }
-    if (threadIdx.x == 0) {
+    if (warp == 0) {
       double s = 0.0;
-      for (int t = 0; t < d; ++t) s = fma(vi[t], vi[t], s);
-      snorm = sqrt(s);
+      for (int t = lane; t < d; t += 32) s = fma(vi[t], vi[t], s);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) snorm = sqrt(s);
     }
     __syncthreads();
     for (int t = threadIdx.x; t < d; t += blockDim.x) vi[t] /= snorm;
@@ -301,9 +329,22 @@ __global__ void __launch_bounds__(256)
   for (int i = threadIdx.x; i < d; i += blockDim.x) {
     const int r = blk * d + i;
     if (r >= M) continue;
-    const double* rr = R + ((size_t)h * M + r) * d;
     double s = 0.0;
-    for (int t = 0; t < d; ++t) s = fma(rr[t], rr[t], s);
+    if (seeded) {
+      const long long nr = NG + ((long long)h * M + r) * d;
+      for (long long gq = nr / 4; gq <= (nr + d - 1) / 4; ++gq) {
+        double z[4];
+        rng::normals4(seed, (uint64_t)gq, z);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const long long n = 4 * gq + p;
+          if (n >= nr && n < nr + d) s = fma(z[p], z[p], s);
+        }
+      }
+    } else {
+      const double* rr = R + ((size_t)h * M + r) * d;
+      for (int t = 0; t < d; ++t) s = fma(rr[t], rr[t], s);
+    }
     dots[i] = sqrt(s);
   }
   __syncthreads();

@@ -115,3 +115,19 @@ def test_decode_init_validation():
     assert F.lib().favor_decode_init(vp(20), 1, 1, 64, 64, 0, None) == -2
     assert F.lib().favor_decode_init(vp(32), 1, 1, 64, 64, 5, None) == -4
     assert F.lib().favor_decode_init(vp(32), 1, 1, 40, 64, 0, None) == -5
+
+
+def test_seeded_orf_validation_rejects_before_any_cuda_call():
+    vp, u = ctypes.c_void_p, ctypes.c_uint64
+    L = F.lib()
+    assert L.favor_orf_omega_seeded(u(1), vp(0), 1, 64, 64, 0, None) == -1
+    assert L.favor_orf_omega_seeded(u(1), vp(24), 1, 64, 64, 0, None) == -2
+    assert L.favor_orf_omega_seeded(u(1), vp(32), 0, 64, 64, 0, None) == -3
+    assert L.favor_orf_omega_seeded(u(1), vp(32), 1, 64, 256, 0, None) == -5
+    assert L.favor_orf_omega_seeded(u(1), vp(32), 1, 64, 64, 3, None) == -5
+    assert L.favor_orf_gaussians_seeded(u(1), vp(32), vp(0), 1, 64, 64, None) == -1
+    assert L.favor_orf_gaussians_seeded(u(1), vp(32), vp(40), 1, 64, 64, None) == -2
+    assert L.favor_orf_gaussians_seeded(u(1), vp(32), vp(48), 1, -1, 64, None) == -3
+    assert L.favor_philox4x64(u(1), u(0), u(4), vp(0), None) == -1
+    assert L.favor_philox4x64(u(1), u(0), u(4), vp(8), None) == -2
+    assert L.favor_philox4x64(u(1), u(0), u(0), vp(16), None) == -3
