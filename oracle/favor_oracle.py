@@ -358,6 +358,68 @@ def favor_rows_head(q, k, v, Om, kind, causal, rows):
     return out
 
 
+# ---------------------------------------------------------------- backward (gradients)
+def phi_vjp(X, Om, kind, dphi):
+    """Gradient with respect to X [L, d] of sum(dphi * phi(X, Om)): the feature map's
+    vector-Jacobian product, row by row.
+
+    Trig, phi = g(x) [cos u, sin u] with u = Omega x and g = exp(|x|^2/2)/sqrt(M):
+        dx = x (dphi . phi) + g Omega^T (-dphi_cos * sin u + dphi_sin * cos u).
+    ReLU, phi = max(u, 0)/sqrt(M):  dx = Omega^T (dphi * [u > 0]) / sqrt(M).
+    """
+    U = X @ Om.T
+    M = Om.shape[0]
+    if kind == TRIG:
+        g = np.exp(0.5 * np.sum(X * X, axis=1)) / np.sqrt(M)
+        dc, ds = dphi[:, :M], dphi[:, M:]
+        return X * np.sum(dphi * phi_trig(X, Om), axis=1)[:, None] + g[:, None] * ((-dc * np.sin(U) + ds * np.cos(U)) @ Om)
+    if kind == RELU:
+        return ((dphi * (U > 0)) @ Om) / np.sqrt(M)
+    raise ValueError(f"unknown feature kind {kind}")
+
+
+def favor_backward_head(q, k, v, Om, kind, causal, dout):
+    """Gradients (dq, dk, dv) of sum(dout * out) for one head, out = FAVOR(q, k, v).
+
+    The definition differentiated is the quadratic form D^-1 A V with A = phi(Q) phi(K)^T
+    (masked to j <= i when causal) ([EXPL, 核心机制]). The linear-time form computes the same out.
+    Reverse mode:
+        dN = dout / D,  dD = -(dout . out) / D            (rows with D = 0 give out = 0: no gradient)
+        dA = dN V^T + dD 1^T  (masked)
+        dphi(Q) = dA phi(K),  dphi(K) = dA^T phi(Q),  dV = A^T dN
+    then each phi through phi_vjp. Omega is a fixed random draw and gets no gradient.
+    """
+    fq, fk = phi(q, Om, kind), phi(k, Om, kind)
+    A = fq @ fk.T
+    if causal:
+        A = np.where(np.arange(k.shape[0])[None, :] <= np.arange(q.shape[0])[:, None], A, 0.0)
+    N, D = A @ v, A.sum(axis=1)
+    out = _normalise(N, D)
+    nz = D != 0.0
+    dN = np.zeros_like(N)
+    dD = np.zeros_like(D)
+    dN[nz] = dout[nz] / D[nz, None]
+    dD[nz] = -np.sum(dout[nz] * out[nz], axis=1) / D[nz]
+    dA = dN @ v.T + dD[:, None]
+    if causal:
+        dA = np.where(np.arange(k.shape[0])[None, :] <= np.arange(q.shape[0])[:, None], dA, 0.0)
+    dq = phi_vjp(q, Om, kind, dA @ fk)
+    dk = phi_vjp(k, Om, kind, dA.T @ fq)
+    return dq, dk, A.T @ dN
+
+
+def favor_backward(Q, K, V, Om, kind, causal, dO):
+    """favor_backward_head over [B, H, L, d]: returns (dQ, dK, dV)."""
+    B, H = Q.shape[:2]
+    res = [np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)]
+    for b in range(B):
+        for h in range(H):
+            g = favor_backward_head(Q[b, h], K[b, h], V[b, h], Om[h], kind, causal, dO[b, h])
+            for r, x in zip(res, g):
+                r[b, h] = x
+    return tuple(res)
+
+
 # ---------------------------------------------------------------- decode: one token per call
 def favor_decode_state(M, dv, kind):
     """An empty carried state (S [F, dv], z [F]) for one head; F = 2M (trig) or M (ReLU)."""

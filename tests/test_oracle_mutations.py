@@ -110,6 +110,29 @@ def _normals_cos_twice(seed, group):
     return out
 
 
+def _backward_no_normaliser_term(q, k, v, Om, kind, causal, dout):
+    fq, fk = O.phi(q, Om, kind), O.phi(k, Om, kind)
+    A = fq @ fk.T
+    if causal:
+        A = np.tril(A)
+    D = A.sum(axis=1)
+    dN = dout / D[:, None]
+    dA = dN @ v.T
+    if causal:
+        dA = np.tril(dA)
+    return O.phi_vjp(q, Om, kind, dA @ fk), O.phi_vjp(k, Om, kind, dA.T @ fq), A.T @ dN
+
+
+def _phi_vjp_no_radial_term(X, Om, kind, dphi):
+    U = X @ Om.T
+    M = Om.shape[0]
+    if kind == O.TRIG:
+        g = np.exp(0.5 * np.sum(X * X, axis=1)) / np.sqrt(M)
+        dc, ds = dphi[:, :M], dphi[:, M:]
+        return g[:, None] * ((-dc * np.sin(U) + ds * np.cos(U)) @ Om)
+    return ((dphi * (U > 0)) @ Om) / np.sqrt(M)
+
+
 CASES = [
     ("phi_trig", _phi_trig_no_exp, [P.test_trig_self_inner_product_identity]),
     ("phi_trig", _phi_trig_cos_twice, [P.test_trig_self_inner_product_identity]),
@@ -123,6 +146,9 @@ CASES = [
     ("softmax_attention_head", _softmax_mask_slip, [lambda: P.test_softmax_matches_torch(True)]),
     ("philox4x64_10", _philox_wrong_weyl, [lambda: P.test_philox_matches_numpy_bit_generator(5, 0)]),
     ("philox_normals", _normals_cos_twice, [P.test_philox_normals_box_muller_form]),
+    ("favor_backward_head", _backward_no_normaliser_term,
+     [lambda: P.test_backward_matches_central_differences(O.RELU, False)]),
+    ("phi_vjp", _phi_vjp_no_radial_term, [lambda: P.test_backward_matches_autograd_of_the_quadratic_form(O.TRIG, True)]),
     ("favor_decode_step_head", _decode_read_before_add,
      [lambda: P.test_decode_steps_equal_masked_rows(O.TRIG)]),
     ("favor_decode_step_head", _decode_value_for_key,

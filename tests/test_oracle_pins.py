@@ -227,6 +227,75 @@ def test_seeded_orf_gaussians_layout():
     assert np.array_equal(G, O.seeded_orf_gaussians(seed, H, M, d)[0])
 
 
+# ------------------------------------------------------------------ backward
+def _loss(q, k, v, om, kind, causal, dout):
+    return float(np.sum(dout * O.favor_explicit_head(q, k, v, om, kind, causal)))
+
+
+@pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_matches_central_differences(kind, causal):
+    # every coordinate of q, k and v, central differences of sum(dout * out) in fp64
+    L, d, M = 10, 4, 8
+    q, k, v = _qkv(L, d, seed=4)
+    om = _orf(M, d, seed=4)[0]
+    dout = np.random.default_rng(8).standard_normal((L, d))
+    g = O.favor_backward_head(q, k, v, om, kind, causal, dout)
+    h = 1e-6
+    for which, x in enumerate((q, k, v)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            fd[idx] = (_loss(*args_p, om, kind, causal, dout) - _loss(*args_m, om, kind, causal, dout)) / (2 * h)
+        np.testing.assert_allclose(g[which], fd, rtol=1e-5, atol=1e-6 * np.abs(fd).max())
+
+
+@pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_matches_autograd_of_the_quadratic_form(kind, causal):
+    # torch autograd (fp64) through the quadratic form written with torch ops
+    L, d, M = 40, 8, 16
+    q, k, v = _qkv(L, d, seed=6)
+    om = _orf(M, d, seed=6)[0]
+    dout = np.random.default_rng(9).standard_normal((L, d))
+    T = [torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v)]
+    W = torch.tensor(om, dtype=torch.float64)
+
+    def feats(X):
+        U = X @ W.T
+        if kind == O.TRIG:
+            g = torch.exp(0.5 * (X * X).sum(dim=1, keepdim=True)) / math.sqrt(M)
+            return g * torch.cat([torch.cos(U), torch.sin(U)], dim=1)
+        return torch.relu(U) / math.sqrt(M)
+
+    A = feats(T[0]) @ feats(T[1]).T
+    if causal:
+        A = torch.tril(A)
+    out = (A @ T[2]) / A.sum(dim=1, keepdim=True)
+    (out * torch.tensor(dout)).sum().backward()
+    for mine, t in zip(O.favor_backward_head(q, k, v, om, kind, causal, dout), T):
+        np.testing.assert_allclose(mine, t.grad.numpy(), rtol=1e-9, atol=1e-12 * np.abs(t.grad.numpy()).max())
+
+
+def test_backward_of_constant_v_has_no_q_or_k_gradient():
+    # out_i = c for every row whatever the weights, so dq = dk = 0 and dv sums dout
+    L, d, M = 30, 8, 16
+    q, k, _ = _qkv(L, d, seed=2)
+    v = np.tile(np.linspace(-1, 1, d), (L, 1))
+    om = _orf(M, d, seed=2)[0]
+    dout = np.random.default_rng(1).standard_normal((L, d))
+    for kind in (O.TRIG, O.RELU):
+        dq, dk, dv = O.favor_backward_head(q, k, v, om, kind, False, dout)
+        assert np.abs(dq).max() < 1e-9 * np.abs(dout).max() and np.abs(dk).max() < 1e-9 * np.abs(dout).max()
+        # rows of A / D sum to one, so sum_j dv_j = sum_i dout_i
+        np.testing.assert_allclose(dv.sum(axis=0), dout.sum(axis=0), rtol=1e-9)
+
+
 # ------------------------------------------------------------------ invariants
 @pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
 @pytest.mark.parametrize("causal", [False, True])
