@@ -349,6 +349,47 @@ def run_orf(args):
                           "blocks": H * (-(-M // d)), "dtype": "bf16 out, fp64 Gram-Schmidt"}), flush=True)
 
 
+def run_backward(args):
+    """fp32 backward (dq, dk, dv) at B=4, H=8, L=4096, d=64, M=256, each variant: microseconds
+    per call and FLOP/s of the algorithmic work, against the fp32 CUDA-core peak."""
+    import torch
+
+    import favor_inputs as fi
+    import linear_kernelized_attention_b200 as F
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    W = WORKLOAD
+    B, H, L, d, M = W["B"], W["H"], W["L"], W["d"], W["M"]
+    q, k, v = (fi.round_to(x, "f32").to(dev) for x in fi.qkv(B, H, L, d, seed=2))
+    dO = torch.randn(B, H, L, d, device=dev, generator=torch.Generator(device=dev).manual_seed(3))
+    G, R = fi.orf_gaussians(H, M, d, seed=2)
+    om = F.favor_orf_omega(torch.from_numpy(G).to(dev), torch.from_numpy(R).to(dev), M, dtype=torch.float32)
+    for name, kind, causal in VARIANTS:
+        for _ in range(max(args.warmup, 3)):
+            F.favor_attention_backward_f32(q, k, v, om, dO, feature_kind=kind, causal=causal, stream=stream)
+        torch.cuda.synchronize()
+        n = 5
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            F.favor_attention_backward_f32(q, k, v, om, dO, feature_kind=kind, causal=causal, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if F.favor_sync_status(stream) != 0:
+            raise RuntimeError("device status not OK")
+        us = 1e3 * a.elapsed_time(b) / n
+        Fe = 2 * M if kind == 0 else M
+        # algorithmic FLOP per head-token: forward projections and state (recomputed) + the
+        # backward's: q and k projections and their transposes, g, h, dv, R and S (2 F (d+1) each)
+        flops = (4 * d * M + 4 * Fe * (d + 1)) + (4 * d * M + 4 * d * M + 10 * Fe * (d + 1))
+        tf = flops * B * H * L / (us * 1e-6) / 1e12
+        print(json.dumps({"backward": True, "variant": name, "B": B, "H": H, "L": L, "d": d, "M": M,
+                          "dtype": "f32", "us_per_call": us, "tokens_per_s": B * H * L / (us * 1e-6),
+                          "algorithmic_tflops": tf}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -363,7 +404,10 @@ def main():
     ap.add_argument("--decode-batches", default="512,4", help="batch sizes B for --decode (H=8)")
     ap.add_argument("--decode-kinds", default="trig,relu", help="feature maps for --decode")
     ap.add_argument("--orf", action="store_true", help="time Omega redrawn on the device from a seed")
+    ap.add_argument("--backward", action="store_true", help="time the fp32 backward pass")
     args = ap.parse_args()
+    if args.backward:
+        return run_backward(args)
     if args.orf:
         return run_orf(args)
     if args.lsweep:

@@ -193,6 +193,25 @@ int favor_attention_f32_noalloc(const float* q, const float* k, const float* v, 
 size_t favor_noalloc_scratch_bytes(void);
 
 /*
+ * fp32 backward pass: the gradients dq, dk, dv of sum(dout * out), out = favor_attention_f32 of
+ * the same arguments. The differentiated quantity is D^-1 A V with A = phi(Q) phi(K)^T (masked
+ * to j <= i when causal), as the explainer's 核心机制 section defines it; it is computed in
+ * linear time, with the causal gradients as reverse prefix sums over 64-token chunks. Omega is
+ * a fixed random draw and gets no gradient. Rows whose denominator is zero (output zero) pass no
+ * gradient.
+ * q, k, v, dout, dq, dk, dv: device float [B, H, L, d]; omega: device float [H, M, d]; all
+ * 16-byte aligned. dq, dk, dv are written in full.
+ * Arithmetic: fp32 on CUDA cores, sin/cos/exp in double rounded to fp32. Feature scale
+ * factors that cancel (exp(|q|^2/2), the key stabiliser, 1/sqrt(M)) are dropped.
+ * Scratch: 2 B H ceil(L/64) F (d+1) + B H L (d+1) + B H floats from the library's stream-ordered
+ * pool on `stream`.
+ * Supported: 1 <= d <= 64, 1 <= M <= 512, L >= 1, B*H <= 65535, ceil(L/64) <= 65535.
+ */
+int favor_attention_backward_f32(const float* q, const float* k, const float* v, const float* omega,
+                                 const float* dout, float* dq, float* dk, float* dv, int B, int H, int L, int d,
+                                 int M, int feature_kind, int causal, void* stream);
+
+/*
  * Causal decode: one token per (batch, head) per call, against a carried state.
  * The explainer's 核心机制 section: the causal prefix sums S_t = S_{t-1} + phi(k_t) v_t^T and
  * z_t = z_{t-1} + phi(k_t), read by the same token's query: out_t = phi(q_t) S_t / phi(q_t) z_t.

@@ -9,7 +9,7 @@ Entry points mirror the C ABI in include/favor.h:
     favor_attention_host, favor_sync_status, favor_status_string, favor_workspace_bytes,
     favor_selftest_timeout, favor_attention_f32_noalloc, favor_noalloc_scratch_bytes,
     favor_decode_state_bytes, favor_decode_init, favor_decode_step, favor_orf_omega_seeded,
-    favor_orf_gaussians_seeded, favor_philox4x64
+    favor_orf_gaussians_seeded, favor_philox4x64, favor_attention_backward_f32
 """
 from __future__ import annotations
 
@@ -44,6 +44,7 @@ _SIGS = {
     "favor_orf_omega_seeded": (_i, [_u64, _vp] + [_i] * 4 + [_vp]),
     "favor_orf_gaussians_seeded": (_i, [_u64, _vp, _vp] + [_i] * 3 + [_vp]),
     "favor_philox4x64": (_i, [_u64, _u64, _u64, _vp, _vp]),
+    "favor_attention_backward_f32": (_i, [_vp] * 8 + [_i] * 7 + [_vp]),
 }
 _LIB = None
 
@@ -296,3 +297,18 @@ def favor_philox4x64(key, first_counter, n_blocks, device="cuda", stream=None):
                                 out.data_ptr(), _stream(stream))
     _check(rc, "favor_philox4x64")
     return out
+
+
+# ---------------------------------------------------------------- backward
+def favor_attention_backward_f32(q, k, v, omega, dout, feature_kind=FAVOR_TRIG, causal=False, stream=None):
+    """fp32 gradients (dq, dk, dv) of sum(dout * out) for out = favor_attention_f32(q, k, v, omega)."""
+    import torch
+    B, H, L, d, M = _check_qkv(q, k, v, omega, torch.float32)
+    if dout.shape != q.shape or dout.dtype != torch.float32 or not dout.is_cuda or not dout.is_contiguous():
+        raise ValueError("dout must be a contiguous float32 CUDA tensor shaped like q")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    rc = lib().favor_attention_backward_f32(q.data_ptr(), k.data_ptr(), v.data_ptr(), omega.data_ptr(),
+                                            dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                            B, H, L, d, M, int(feature_kind), int(causal), _stream(stream))
+    _check(rc, "favor_attention_backward_f32")
+    return dq, dk, dv

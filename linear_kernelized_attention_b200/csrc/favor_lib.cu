@@ -17,6 +17,7 @@
 #include "kernel_bidir.cuh"
 #include "kernel_causal.cuh"
 #include "kernel_decode.cuh"
+#include "kernels_bwd_f32.cuh"
 
 namespace favor {
 
@@ -419,6 +420,56 @@ int launch_orf(const double* G, const double* R, void* omega, int H, int M, int 
   return cudaGetLastError() == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ fp32 backward
+size_t bwd_workspace(int BH, int L, int d, int M, int kind) {
+  const size_t F = kind == FAVOR_TRIG ? 2 * (size_t)M : (size_t)M;
+  const size_t nch = (L + f32::kChunk - 1) / f32::kChunk;
+  return (2 * (size_t)BH * nch * F * (d + 1) + (size_t)BH * L * (d + 1) + BH) * sizeof(float);
+}
+
+// cmax (trig) -> chunk states of phi(K)[V|1] and their scan (S) -> k_bwd_query (dq, e, R shares)
+// -> reverse scan of R -> k_bwd_key (dk, dv). Scratch from the stream-ordered pool.
+int launch_bwd_f32(const float* q, const float* k, const float* v, const float* omega, const float* dout,
+                   float* dq, float* dk, float* dv, int B, int H, int L, int d, int M, int kind, int causal,
+                   cudaStream_t st) {
+  const int BH = B * H;
+  const int F = kind == FAVOR_TRIG ? 2 * M : M;
+  const int nch = (L + f32::kChunk - 1) / f32::kChunk;
+  const int nft = (F + f32::kFeatTile - 1) / f32::kFeatTile;
+  if (BH > 65535 || nch > 65535) return FAVOR_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  int rc = scratch_alloc(&ws, bwd_workspace(BH, L, d, M, kind), st);
+  if (rc != FAVOR_OK) return rc;
+  const size_t per = (size_t)BH * nch * F * (d + 1);
+  float* dS = static_cast<float*>(ws);
+  float* Rc = dS + per;
+  float* E = Rc + per;
+  float* cmax = E + (size_t)BH * L * (d + 1);
+  const size_t sm_state = (size_t)(2 * f32::kChunk * d + f32::kChunk + f32::kChunk * f32::kFeatTile) * 4;
+  const size_t sm_bwd = (size_t)bwd::bwd_smem(d).total * 4;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(f32::k_chunk_state), (int)sm_state) != FAVOR_OK ||
+      ensure_smem_attr(reinterpret_cast<const void*>(bwd::k_bwd_query), (int)sm_bwd) != FAVOR_OK ||
+      ensure_smem_attr(reinterpret_cast<const void*>(bwd::k_bwd_key), (int)sm_bwd) != FAVOR_OK)
+    rc = FAVOR_ERR_CUDA;
+  if (rc == FAVOR_OK) {
+    if (kind == FAVOR_TRIG) f32::k_key_halfnorm_max<<<BH, f32::kThreads, 0, st>>>(k, cmax, L, d);
+    f32::k_chunk_state<<<dim3(nft, nch, BH), f32::kThreads, sm_state, st>>>(k, v, omega, cmax, dS, H, L, d, M,
+                                                                             F, kind);
+    const long long per_chunk = (long long)F * (d + 1);
+    const long long total = (long long)BH * per_chunk;
+    const unsigned sblocks = (unsigned)((total + 255) / 256);
+    f32::k_scan_chunks<<<sblocks, 256, 0, st>>>(dS, nch, per_chunk, total, causal);
+    bwd::k_bwd_query<<<dim3(nch, BH), bwd::kThreads, sm_bwd, st>>>(q, k, v, omega, cmax, dS, dout, dq, E, Rc, H,
+                                                                   L, d, M, F, kind, causal);
+    bwd::k_scan_chunks_rev<<<sblocks, 256, 0, st>>>(Rc, nch, per_chunk, total, causal);
+    bwd::k_bwd_key<<<dim3(nch, BH), bwd::kThreads, sm_bwd, st>>>(q, k, v, omega, cmax, Rc, E, dk, dv, H, L, d,
+                                                                 M, F, kind, causal);
+    if (cudaGetLastError() != cudaSuccess) rc = FAVOR_ERR_CUDA;
+  }
+  cudaFreeAsync(ws, st);
+  return rc;
+}
+
 // ====================================================================== C ABI
 extern "C" {
 
@@ -578,6 +629,19 @@ int favor_attention_f32_noalloc(const float* q, const float* k, const float* v, 
 }
 
 size_t favor_noalloc_scratch_bytes(void) { return favor::kNoAllocScratchBytes; }
+
+int favor_attention_backward_f32(const float* q, const float* k, const float* v, const float* omega,
+                                 const float* dout, float* dq, float* dk, float* dv, int B, int H, int L, int d,
+                                 int M, int feature_kind, int causal, void* stream) {
+  int rc = check_common(q, k, v, omega, dout, B, H, L, d, M, feature_kind);
+  if (rc != FAVOR_OK) return rc;
+  if (!dq || !dk || !dv) return FAVOR_ERR_NULL;
+  if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return FAVOR_ERR_ALIGN;
+  if (d > bwd::kMaxD || M > 512) return FAVOR_ERR_UNSUPPORTED;
+  if ((rc = check_device()) != FAVOR_OK) return rc;
+  return launch_bwd_f32(q, k, v, omega, dout, dq, dk, dv, B, H, L, d, M, feature_kind, causal,
+                        static_cast<cudaStream_t>(stream));
+}
 
 size_t favor_decode_state_bytes(int B, int H, int d, int M, int feature_kind) {
   if (check_decode(nullptr, B, H, d, M, feature_kind) != FAVOR_OK) return 0;

@@ -408,6 +408,47 @@ def favor_backward_head(q, k, v, Om, kind, causal, dout):
     return dq, dk, A.T @ dN
 
 
+def backward_magnitudes_head(q, k, v, Om, kind, causal, dout):
+    """Rounding scales of the gradients: the reverse pass of favor_backward_head with every
+    factor replaced by its absolute value (|phi|, |V|, |dout|, |out|, |1/D|, |sin|, |cos|, |x|).
+
+    Each gradient element is a sum of products; a finite-precision evaluation of it errs by at
+    most a small multiple of the unit roundoff times the sum of the products' absolute values,
+    which is what this returns (dq_abs, dk_abs, dv_abs). A gradient that cancels (row 0 of a
+    causal head has dq = 0 exactly, its output being v_0 whatever q_0 is) keeps a non-zero
+    scale here.
+    """
+    fq, fk = np.abs(phi(q, Om, kind)), np.abs(phi(k, Om, kind))
+    A = fq @ fk.T
+    Aphi = phi(q, Om, kind) @ phi(k, Om, kind).T
+    if causal:
+        mask = np.arange(k.shape[0])[None, :] <= np.arange(q.shape[0])[:, None]
+        A, Aphi = np.where(mask, A, 0.0), np.where(mask, Aphi, 0.0)
+    D = Aphi.sum(axis=1)
+    out = _normalise(Aphi @ v, D)
+    nz = D != 0.0
+    dN = np.zeros((q.shape[0], v.shape[1]))
+    dD = np.zeros(q.shape[0])
+    dN[nz] = np.abs(dout[nz]) / np.abs(D[nz, None])
+    dD[nz] = np.sum(np.abs(dout[nz] * out[nz]), axis=1) / np.abs(D[nz])
+    dA = dN @ np.abs(v).T + dD[:, None]
+    if causal:
+        dA = np.where(mask, dA, 0.0)
+
+    def jac_abs(X, dphi):
+        U = X @ Om.T
+        M = Om.shape[0]
+        aO = np.abs(Om)
+        if kind == TRIG:
+            g = np.exp(0.5 * np.sum(X * X, axis=1)) / np.sqrt(M)
+            dc, ds = dphi[:, :M], dphi[:, M:]
+            radial = np.abs(X) * np.sum(dphi * np.abs(phi_trig(X, Om)), axis=1)[:, None]
+            return radial + g[:, None] * ((dc * np.abs(np.sin(U)) + ds * np.abs(np.cos(U))) @ aO)
+        return ((dphi * (U > 0)) @ aO) / np.sqrt(M)
+
+    return jac_abs(q, dA @ fk), jac_abs(k, dA.T @ fq), A.T @ dN
+
+
 def favor_backward(Q, K, V, Om, kind, causal, dO):
     """favor_backward_head over [B, H, L, d]: returns (dQ, dK, dV)."""
     B, H = Q.shape[:2]

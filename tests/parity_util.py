@@ -43,3 +43,34 @@ def check_rows(got, ref, cond, tol, u, label=""):
     }
     assert stats["bad"] == 0, f"{label}: {stats}"
     return stats
+
+
+def check_grads(got, ref, mags, cond, tol, u, label=""):
+    """Backward metric for one head.
+
+    got and ref are (dq, dk, dv) [L, d]. mags are the oracle's rounding scales
+    (backward_magnitudes_head): each element's sum of absolute products. cond [L] holds the
+    forward row condition numbers. Row r of each gradient passes if
+        max_t |g - o|  <=  tol max_t |o_r|  +  u (max_t mag_r + c_r max_t |o_r|)
+    - c_r = cond_r for dq, and the head's worst cond for dk and dv, since every query row feeds
+      them.
+    - The magnitude term bounds the rounding of the gradient's own sums. A row that cancels to
+      zero (row 0 of a causal head) keeps that allowance and nothing more.
+    - The cond term carries the rounding of the denominator the gradient divides by.
+    """
+    cond = np.nan_to_num(np.asarray(cond, dtype=np.float64), nan=np.inf, posinf=np.inf)
+    worst = float(np.max(cond[np.isfinite(cond)])) if np.any(np.isfinite(cond)) else np.inf
+    stats = {}
+    for name, g, o, m, c in (("dq", got[0], ref[0], mags[0], cond), ("dk", got[1], ref[1], mags[1], worst),
+                             ("dv", got[2], ref[2], mags[2], worst)):
+        g, o, m = (np.asarray(x, dtype=np.float64) for x in (g, o, m))
+        assert np.all(np.isfinite(g)), f"{label}: non-finite {name}"
+        err = np.abs(g - o).max(axis=1)
+        on = np.abs(o).max(axis=1)
+        allowed = tol * on + u * (m.max(axis=1) + c * on)
+        ratio = np.where(allowed > 0, err / np.where(allowed > 0, allowed, 1.0), np.where(err > 0, np.inf, 0.0))
+        r = int(np.argmax(ratio))
+        stats[name] = {"max_over_allowed": float(ratio[r]), "row": r,
+                       "rel_at_row": float(err[r] / on[r]) if on[r] > 0 else float(err[r])}
+        assert np.all(ratio <= 1.0), f"{label}: {name} {stats}"
+    return stats

@@ -131,3 +131,20 @@ def test_seeded_orf_validation_rejects_before_any_cuda_call():
     assert L.favor_philox4x64(u(1), u(0), u(4), vp(0), None) == -1
     assert L.favor_philox4x64(u(1), u(0), u(4), vp(8), None) == -2
     assert L.favor_philox4x64(u(1), u(0), u(0), vp(16), None) == -3
+
+
+def test_backward_validation_rejects_before_any_cuda_call():
+    vp = ctypes.c_void_p
+    L = F.lib()
+
+    def call(**over):
+        a = dict(q=16, k=32, v=48, om=64, do=80, dq=96, dk=112, dv=128, B=1, H=1, L_=8, d=64, M=64, kind=0)
+        a.update(over)
+        return L.favor_attention_backward_f32(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["om"]), vp(a["do"]),
+                                              vp(a["dq"]), vp(a["dk"]), vp(a["dv"]), a["B"], a["H"], a["L_"],
+                                              a["d"], a["M"], a["kind"], 0, None)
+    assert call(do=0) == -1 and call(dk=0) == -1
+    assert call(dv=136) == -2 and call(q=20) == -2
+    assert call(L_=0) == -3
+    assert call(kind=2) == -4
+    assert call(d=65) == -5 and call(M=513) == -5

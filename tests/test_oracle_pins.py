@@ -296,6 +296,40 @@ def test_backward_of_constant_v_has_no_q_or_k_gradient():
         np.testing.assert_allclose(dv.sum(axis=0), dout.sum(axis=0), rtol=1e-9)
 
 
+@pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_magnitudes_bound_perturbed_gradients(kind, causal):
+    # the magnitudes dominate the gradients, and a relative perturbation of size eps on every
+    # factor (features, V, dout) moves the gradients by at most a few eps times them
+    L, d, M = 24, 8, 16
+    q, k, v = _qkv(L, d, seed=12)
+    om = _orf(M, d, seed=12)[0]
+    dout = np.random.default_rng(13).standard_normal((L, d))
+    g = O.favor_backward_head(q, k, v, om, kind, causal, dout)
+    mags = O.backward_magnitudes_head(q, k, v, om, kind, causal, dout)
+    cond = O.row_condition_head(q, k, v, om, kind, causal)
+    for a, m in zip(g, mags):
+        assert np.all(np.abs(a) <= m * (1 + 1e-12) + 1e-300)
+    eps = 1e-7
+    rng = np.random.default_rng(14)
+    base_phi = O.phi
+    orig = O.phi
+
+    def noisy(X, Om, kd):
+        f = base_phi(X, Om, kd)
+        return f * (1 + eps * rng.uniform(-1, 1, f.shape))
+    try:
+        O.phi = noisy
+        gp = O.favor_backward_head(q, k, v * (1 + eps * rng.uniform(-1, 1, v.shape)), om, kind, causal,
+                                   dout * (1 + eps * rng.uniform(-1, 1, dout.shape)))
+    finally:
+        O.phi = orig
+    # first order: the change is bounded by eps (magnitudes + cond * |gradient|), up to a small factor
+    worst = max(float(cond[np.isfinite(cond)].max()), 1.0)
+    for a, b, m in zip(g, gp, mags):
+        assert np.all(np.abs(a - b) <= 20 * eps * (m + worst * np.abs(a).max()))
+
+
 # ------------------------------------------------------------------ invariants
 @pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
 @pytest.mark.parametrize("causal", [False, True])
