@@ -175,6 +175,24 @@ def oracle_sample(seconds, per_step=False):
     return tokens / dt, dt, heads
 
 
+def oracle_timed(fn, seconds):
+    """Call fn() (one unit of oracle work, returning the units it did) until `seconds` have
+    passed; returns (units per second, seconds, calls)."""
+    units, calls, t0 = 0, 0, time.perf_counter()
+    while True:
+        units += fn()
+        calls += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return units / dt, dt, calls
+
+
+def fp32_alu_peak_tflops(sm_mhz=1965.0, sms=148):
+    """fp32 CUDA-core peak: 128 FMA lanes per SM, 2 FLOP each, at the given clock."""
+    return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
 def run_reference(args, rank):
     if rank != 0:
         return
@@ -310,8 +328,25 @@ def run_decode(args):
             us = 1e3 * a.elapsed_time(b) / (reps * T)
             nb = decode_bytes_per_call(B, H, d, M, kind)
             gbs = nb / (us * 1e-6) / 1e9
+            cpu = None
+            if not args.no_cpu_baseline and B == batches[0]:
+                import numpy as np
+
+                from oracle import favor_oracle as O
+                qh, kh, vh = (fi.as_f64(x[:, 0, 0].cpu()) for x in (q, k, v))
+                omh = fi.as_f64(omega[0].cpu())
+                S0, z0 = O.favor_decode_state(M, d, kind)
+
+                def one_head():
+                    for t in range(T):
+                        O.favor_decode_step_head(S0, z0, qh[t], kh[t], vh[t], omh, kind)
+                    return T
+                r, dt, calls = oracle_timed(one_head, 5.0)
+                cpu = {"value": r, "unit": "head-tokens/s", "cores": blas_threads(), "kind": "oracle",
+                       "sample": f"{calls} x {T} decode steps of one head (favor_decode_step_head), {dt:.1f} s"}
             print(json.dumps({
                 "decode": True, "variant": "trig" if kind == 0 else "relu", "B": B, "H": H, "d": d, "M": M,
+                "cpu_baseline": cpu,
                 "us_per_call": us, "tokens_per_s": B * H / (us * 1e-6),
                 "state_mb": F.favor_decode_state_bytes(B, H, d, M, kind) / 1e6,
                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
@@ -345,8 +380,20 @@ def run_orf(args):
         if F.favor_sync_status(stream) != 0:
             raise RuntimeError("device status not OK")
         us = 1e3 * a.elapsed_time(b) / n
+        cpu = None
+        if not args.no_cpu_baseline and H == 8:
+            from oracle import favor_oracle as O
+
+            def one_head():
+                G, R = O.seeded_orf_gaussians(7, 1, M, d)
+                O.orf_matrices(G, R, M)
+                return 1
+            r, dt, calls = oracle_timed(one_head, 5.0)
+            cpu = {"value": 1e6 / r * H, "unit": "us per call (H heads)", "cores": blas_threads(), "kind": "oracle",
+                   "sample": f"{calls} head(s) of seeded_orf_gaussians + orf_matrices, {dt:.1f} s"}
         print(json.dumps({"orf": True, "H": H, "M": M, "d": d, "us_per_call": us,
-                          "blocks": H * (-(-M // d)), "dtype": "bf16 out, fp64 Gram-Schmidt"}), flush=True)
+                          "blocks": H * (-(-M // d)), "dtype": "bf16 out, fp64 Gram-Schmidt",
+                          "cpu_baseline": cpu}), flush=True)
 
 
 def run_backward(args):
@@ -385,9 +432,24 @@ def run_backward(args):
         # backward's: q and k projections and their transposes, g, h, dv, R and S (2 F (d+1) each)
         flops = (4 * d * M + 4 * Fe * (d + 1)) + (4 * d * M + 4 * d * M + 10 * Fe * (d + 1))
         tf = flops * B * H * L / (us * 1e-6) / 1e12
+        cpu = None
+        if not args.no_cpu_baseline:
+            import numpy as np
+
+            from oracle import favor_oracle as O
+            Lh = 1024
+            qh, kh, vh, dh = (fi.as_f64(x[0, 0, :Lh].cpu()) for x in (q, k, v, dO))
+            omh = fi.as_f64(om[0].cpu())
+            r, dt, calls = oracle_timed(lambda: (O.favor_backward_head(qh, kh, vh, omh, kind, causal, dh), Lh)[1], 4.0)
+            cpu = {"value": r, "unit": "head-tokens/s", "cores": blas_threads(), "kind": "oracle",
+                   "sample": f"{calls} call(s) of favor_backward_head on one head, L={Lh} (quadratic form), {dt:.1f} s"}
+        peak = fp32_alu_peak_tflops()
         print(json.dumps({"backward": True, "variant": name, "B": B, "H": H, "L": L, "d": d, "M": M,
                           "dtype": "f32", "us_per_call": us, "tokens_per_s": B * H * L / (us * 1e-6),
-                          "algorithmic_tflops": tf}), flush=True)
+                          "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                                       "frac": tf / peak,
+                                       "peak_source": "fp32 FMA lanes: 148 SMs x 128 x 2 FLOP x 1965 MHz"},
+                          "cpu_baseline": cpu}), flush=True)
 
 
 def main():
