@@ -1,5 +1,5 @@
 /*
- * favor.h - C ABI of libfavor.so, the B200 (sm_100a) FAVOR attention forward pass.
+ * favor.h - C ABI of libfavor.so: B200 (sm_100a) FAVOR attention.
  *
  * The operation. For each head h and batch b, with Q, K, V in R^{L x d} and Omega_h in R^{M x d}:
  *   out = D_hat^-1 (phi(Q) (phi(K)^T [V | 1]))
@@ -35,9 +35,14 @@
  * favor_sync_status() synchronises the stream and returns the device-side status word.
  *
  * Scratch. The bf16 path needs none (cross-CTA sums travel through distributed shared memory).
- * favor_attention_f32 and favor_attention_host take scratch from a library-owned stream-ordered
- * pool on `stream` and release it on the same stream; favor_attention_f32_noalloc uses a static
- * device array instead.
+ * favor_attention_f32, favor_attention_backward_f32 and favor_attention_host take scratch from a
+ * library-owned stream-ordered pool on `stream` and release it on the same stream;
+ * favor_attention_f32_noalloc uses a static device array instead. The decode step keeps its
+ * state in caller-owned memory and needs no scratch; so does favor_orf_omega_seeded.
+ *
+ * Beyond the forward pass: a causal decode step against a carried state
+ * (favor_decode_*), the fp32 backward pass (favor_attention_backward_f32) and ORF redrawn on
+ * the device from a seed (favor_orf_omega_seeded).
  *
  * Errors. Negative favor_status codes. On an error nothing is launched and no output is
  * written.
