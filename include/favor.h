@@ -68,7 +68,7 @@ typedef enum {
   FAVOR_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned */
   FAVOR_ERR_SHAPE = -3,       /* a size is non-positive or the total overflows */
   FAVOR_ERR_KIND = -4,        /* feature_kind is not FAVOR_TRIG / FAVOR_RELU */
-  FAVOR_ERR_UNSUPPORTED = -5, /* a valid shape this build has no kernel for */
+  FAVOR_ERR_UNSUPPORTED = -5, /* a valid shape the library has no kernel for */
   FAVOR_ERR_CUDA = -6,        /* a CUDA runtime call failed (launch, allocation, copy) */
   FAVOR_ERR_TIMEOUT = -7,     /* a bounded device-side wait gave up */
   FAVOR_ERR_DEVICE = -8       /* the current device is not sm_100 */

@@ -480,7 +480,7 @@ const char* favor_status_string(int status) {
     case FAVOR_ERR_ALIGN: return "a pointer is not 16-byte aligned";
     case FAVOR_ERR_SHAPE: return "a size is non-positive or too large";
     case FAVOR_ERR_KIND: return "feature_kind must be FAVOR_TRIG (0) or FAVOR_RELU (1)";
-    case FAVOR_ERR_UNSUPPORTED: return "shape not supported by this build";
+    case FAVOR_ERR_UNSUPPORTED: return "shape not supported by the library";
     case FAVOR_ERR_CUDA: return "a CUDA runtime call failed";
     case FAVOR_ERR_TIMEOUT: return "a bounded device-side wait timed out";
     case FAVOR_ERR_DEVICE: return "the current device is not sm_100";
