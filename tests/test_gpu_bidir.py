@@ -34,7 +34,7 @@ def test_bidir_small(kind, B, H, L, M):
     c = Case(B, H, L, 64, M, seed=B * 100 + L + M)
     g = _run(c, kind).reshape(B * H, L, 64)
     ref, cond, _ = c.oracle(kind, False)
-    check_rows(g, ref, cond, TOL_BF16, U_BF16, f"kind={kind} {B}x{H}x{L} M={M}")
+    check_rows(g, ref, cond, TOL_BF16, U_BF16, f"kind={kind} {B}x{H}x{L} M={M}", trig=kind == 0)
 
 
 @pytest.mark.parametrize("kind", [0, 1])
@@ -45,7 +45,7 @@ def test_bidir_many_heads_single_cta_per_head(kind):
     heads = [(0, 0), (0, 79), (1, 40), (1, 79)]
     ref, cond, _ = c.oracle(kind, False, heads=heads)
     sel = np.stack([g[b * 80 + h] for b, h in heads])
-    check_rows(sel, ref, cond, TOL_BF16, U_BF16, f"many heads kind={kind}")
+    check_rows(sel, ref, cond, TOL_BF16, U_BF16, f"many heads kind={kind}", trig=kind == 0)
 
 
 def test_bidir_protein_mlm_shape_trig():
@@ -63,7 +63,7 @@ def test_bidir_bench_workload(kind):
     c = Case(4, 8, 4096, 64, 256, seed=0)
     g = _run(c, kind).reshape(32, 4096, 64)
     ref, cond, _ = c.oracle(kind, False)
-    st = check_rows(g, ref, cond, TOL_BF16, U_BF16, f"bench kind={kind}")
+    st = check_rows(g, ref, cond, TOL_BF16, U_BF16, f"bench kind={kind}", trig=kind == 0)
     print(st)
 
 
@@ -95,7 +95,7 @@ def test_bidir_constant_v_and_zero_queries():
         # the exact answer is the constant row; trig rows with heavy cancellation get the
         # condition-aware allowance like every other parity check
         np.testing.assert_allclose(ref, np.broadcast_to(fi.as_f64(val), ref.shape), rtol=1e-9, atol=1e-9)
-        check_rows(g, ref, cond, TOL_BF16, U_BF16, f"constant v kind={kind}")
+        check_rows(g, ref, cond, TOL_BF16, U_BF16, f"constant v kind={kind}", trig=kind == 0)
     # ReLU with q = 0: every feature of q is 0, so the denominator is 0 and the row is 0
     c.t[0] = torch.zeros_like(c.t[0])
     c._dev = None

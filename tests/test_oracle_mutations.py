@@ -133,7 +133,38 @@ def _phi_vjp_no_radial_term(X, Om, kind, dphi):
     return ((dphi * (U > 0)) @ Om) / np.sqrt(M)
 
 
+def _rows_sorted_order(q, k, v, Om, kind, causal, rows):
+    # cursor slip: rows written in sorted order instead of the asked order
+    rows = np.asarray(rows)
+    ref = O.favor_explicit_head(q, k, v, Om, kind, causal, np.sort(rows))
+    return ref
+
+
+def _rows_read_before_add(q, k, v, Om, kind, causal, rows):
+    # cursor slip: the state is read before key j is added (keys j < i instead of j <= i)
+    rows = np.asarray(rows)
+    fq, fk = O.phi(q[rows], Om, kind), O.phi(k, Om, kind)
+    S, z = np.zeros((fk.shape[1], v.shape[1])), np.zeros(fk.shape[1])
+    out = np.zeros((len(rows), v.shape[1]))
+    order = np.argsort(rows, kind="stable")
+    pos = 0
+    for j in range(q.shape[0]):
+        while pos < len(order) and rows[order[pos]] == j:
+            r = order[pos]
+            den = fq[r] @ z
+            if den != 0.0:
+                out[r] = (fq[r] @ S) / den
+            pos += 1
+        S += np.outer(fk[j], v[j])
+        z += fk[j]
+    if not causal:
+        return O._normalise(fq @ (fk.T @ v), fq @ fk.sum(axis=0))
+    return out
+
+
 CASES = [
+    ("favor_rows_head", _rows_sorted_order, [lambda: P.test_rows_head_equals_explicit_rows(O.TRIG, False)]),
+    ("favor_rows_head", _rows_read_before_add, [lambda: P.test_rows_head_equals_explicit_rows(O.RELU, True)]),
     ("phi_trig", _phi_trig_no_exp, [P.test_trig_self_inner_product_identity]),
     ("phi_trig", _phi_trig_cos_twice, [P.test_trig_self_inner_product_identity]),
     ("phi_trig", _phi_trig_sign_slip, [P.test_trig_cross_term_closed_form]),

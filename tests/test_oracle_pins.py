@@ -134,6 +134,43 @@ def test_causal_prefix_equals_masked(kind):
     np.testing.assert_allclose(cau[-1], O.favor_bidirectional_head(q, k, v, om, kind)[-1], rtol=1e-10)
 
 
+# ------------------------------------------------------------------ sampled rows (the GPU tests' reference)
+def _sample_rows(L, seed):
+    # unsorted, with duplicates, and both ends of the sequence
+    rng = np.random.default_rng(seed)
+    return np.concatenate([[L - 1, 0], rng.integers(0, L, 40), [7, 7, L - 1, 0, 1]])
+
+
+@pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
+@pytest.mark.parametrize("causal", [False, True])
+def test_rows_head_equals_explicit_rows(kind, causal):
+    # favor_rows_head walks the keys once with a cursor over the sorted rows; the explicit
+    # quadratic form D^-1 A V computes each asked row on its own, in the asked order
+    L = 97
+    q, k, v = _qkv(L, 16, seed=61)
+    om = _orf(32, 16, seed=61)[0]
+    rows = _sample_rows(L, 61)
+    got = O.favor_rows_head(q, k, v, om, kind, causal, rows)
+    ref = O.favor_explicit_head(q, k, v, om, kind, causal, rows)
+    assert got.shape == (len(rows), v.shape[1])
+    np.testing.assert_allclose(got, ref, rtol=1e-9, atol=1e-12 * np.abs(ref).max())
+    if causal:
+        np.testing.assert_allclose(got[1], v[0], rtol=1e-12)  # row 0 reads key 0 alone
+    np.testing.assert_allclose(got[0], got[-3], rtol=1e-13)  # duplicated row L-1
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_row_condition_follows_the_asked_rows(causal):
+    # the cursor of row_condition_head: asked rows in any order (duplicates included) give the
+    # same numbers as the full sequence taken at those rows
+    L = 97
+    q, k, v = _qkv(L, 16, seed=62)
+    om = _orf(32, 16, seed=62)[0]
+    rows = _sample_rows(L, 62)
+    full = O.row_condition_head(q, k, v, om, O.TRIG, causal)
+    np.testing.assert_allclose(O.row_condition_head(q, k, v, om, O.TRIG, causal, rows), full[rows], rtol=1e-12)
+
+
 # ------------------------------------------------------------------ decode step (carried state)
 @pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
 def test_decode_steps_equal_masked_rows(kind):
