@@ -186,9 +186,12 @@ int favor_attention_host(const void* q, const void* k, const void* v, const void
  *   Overlap: every call on a device uses the same array. Calls whose executions overlap (on
  *   different streams, or from different host threads without ordering between their streams)
  *   race on it and give undefined results. Order them on one stream or with events.
- *   First call: it looks up the array's device address with cudaGetSymbolAddress, once per
- *   device, and returns FAVOR_ERR_CUDA if that fails. Make a first call on each device before
- *   any stream capture begins.
+ *   Address: every call that is not under stream capture looks up the array's device address
+ *   with cudaGetSymbolAddress (FAVOR_ERR_CUDA if that fails), so a device reset between calls,
+ *   which replaces the context the address belongs to, leaves no stale pointer behind. A call
+ *   under stream capture reuses the address the last uncaptured call on the device found, and
+ *   returns FAVOR_ERR_UNSUPPORTED if there was none: make a first call on each device before any
+ *   stream capture begins, and again after a device reset.
  */
 int favor_attention_f32_noalloc(const float* q, const float* k, const float* v, const float* omega,
                                 float* out, int B, int H, int L, int d, int M, int feature_kind,

@@ -105,6 +105,19 @@ def _check_qkv(q, k, v, omega, dtype):
     return B, H, L, d, omega.shape[1]
 
 
+def _check_out(out, like, name="out"):
+    """An output tensor must match `like` in shape, dtype and device, and be contiguous: the C
+    layer sees only a pointer and writes B*H*L*d elements through it."""
+    import torch
+    if not isinstance(out, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if out.shape != like.shape or out.dtype != like.dtype or out.device != like.device:
+        raise ValueError(f"{name} must have shape {tuple(like.shape)}, dtype {like.dtype} and device "
+                         f"{like.device}; got {tuple(out.shape)}, {out.dtype}, {out.device}")
+    if not out.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
 def favor_attention(q, k, v, omega, out=None, feature_kind=FAVOR_TRIG, causal=False, chunk=0,
                     stream=None):
     """bf16 FAVOR forward on the tensor-core path. q, k, v: [B,H,L,d]; omega: [H,M,d]."""
@@ -112,6 +125,7 @@ def favor_attention(q, k, v, omega, out=None, feature_kind=FAVOR_TRIG, causal=Fa
     B, H, L, d, M = _check_qkv(q, k, v, omega, torch.bfloat16)
     if out is None:
         out = torch.empty_like(q)
+    _check_out(out, q)
     rc = lib().favor_attention_chunked(q.data_ptr(), k.data_ptr(), v.data_ptr(), omega.data_ptr(),
                                        out.data_ptr(), B, H, L, d, M, int(feature_kind), int(causal),
                                        int(chunk), _stream(stream))
@@ -131,11 +145,20 @@ def favor_attention_f32(q, k, v, omega, out=None, feature_kind=FAVOR_TRIG, causa
     B, H, L, d, M = _check_qkv(q, k, v, omega, torch.float32)
     if out is None:
         out = torch.empty_like(q)
+    _check_out(out, q)
     rc = lib().favor_attention_f32(q.data_ptr(), k.data_ptr(), v.data_ptr(), omega.data_ptr(),
                                    out.data_ptr(), B, H, L, d, M, int(feature_kind), int(causal),
                                    _stream(stream))
     _check(rc, "favor_attention_f32")
     return out
+
+
+def _check_omega_out(out, H, M, d):
+    import torch
+    if not isinstance(out, torch.Tensor) or not out.is_cuda or not out.is_contiguous():
+        raise TypeError("out must be a contiguous CUDA tensor")
+    if tuple(out.shape) != (H, M, d) or out.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError(f"out must have shape {(H, M, d)} and dtype float32 or bfloat16")
 
 
 def favor_orf_omega(gauss_blocks, gauss_norms, M, dtype=None, out=None, stream=None):
@@ -150,6 +173,7 @@ def favor_orf_omega(gauss_blocks, gauss_norms, M, dtype=None, out=None, stream=N
             raise TypeError("Gaussian draws must be contiguous float64 CUDA tensors")
     if out is None:
         out = torch.empty((H, M, d), dtype=dtype, device=gauss_blocks.device)
+    _check_omega_out(out, H, M, d)
     code = {torch.float32: 0, torch.bfloat16: 1}[out.dtype]
     rc = lib().favor_orf_omega(gauss_blocks.data_ptr(), gauss_norms.data_ptr(), out.data_ptr(), H, M,
                                d, code, _stream(stream))
@@ -161,10 +185,19 @@ def favor_attention_host(q, k, v, omega, out, feature_kind=FAVOR_TRIG, causal=Fa
     """Host-buffer entry: q, k, v, omega, out are CPU tensors (pinned for async copies)."""
     import torch
     for t in (q, k, v, omega, out):
-        if t.is_cuda or not t.is_contiguous():
+        if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_contiguous():
             raise TypeError("favor_attention_host takes contiguous CPU tensors")
+    if q.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("favor_attention_host takes float32 or bfloat16 tensors")
     code = {torch.float32: 0, torch.bfloat16: 1}[q.dtype]
+    if q.dim() != 4:
+        raise ValueError("q must have shape [B, H, L, d]")
     B, H, L, d = q.shape
+    for name, t in (("k", k), ("v", v), ("out", out)):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError(f"{name} must match q in shape {tuple(q.shape)} and dtype {q.dtype}")
+    if omega.dim() != 3 or omega.shape[0] != H or omega.shape[2] != d or omega.dtype != q.dtype:
+        raise ValueError("omega must have shape [H, M, d] and q's dtype")
     M = omega.shape[1]
     rc = lib().favor_attention_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), omega.data_ptr(),
                                     out.data_ptr(), B, H, L, d, M, int(feature_kind), int(causal),
@@ -194,6 +227,7 @@ def favor_attention_f32_noalloc(q, k, v, omega, out=None, feature_kind=FAVOR_TRI
     B, H, L, d, M = _check_qkv(q, k, v, omega, torch.float32)
     if out is None:
         out = torch.empty_like(q)
+    _check_out(out, q)
     rc = lib().favor_attention_f32_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), omega.data_ptr(),
                                            out.data_ptr(), B, H, L, d, M, int(feature_kind), int(causal),
                                            _stream(stream))
@@ -257,6 +291,7 @@ def favor_decode_step(q, k, v, omega, state, out=None, feature_kind=FAVOR_TRIG, 
         raise ValueError(f"state must be a CUDA tensor of at least {need} bytes")
     if out is None:
         out = torch.empty_like(q)
+    _check_out(out, q)
     rc = lib().favor_decode_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), omega.data_ptr(),
                                  state.data_ptr(), out.data_ptr(), B, H, d, M, int(feature_kind),
                                  _stream(stream))
@@ -271,6 +306,7 @@ def favor_orf_omega_seeded(seed, H, M, d, dtype=None, out=None, device="cuda", s
     dtype = dtype or torch.bfloat16
     if out is None:
         out = torch.empty((H, M, d), dtype=dtype, device=device)
+    _check_omega_out(out, H, M, d)
     code = {torch.float32: 0, torch.bfloat16: 1}[out.dtype]
     rc = lib().favor_orf_omega_seeded(int(seed) & (2**64 - 1), out.data_ptr(), H, M, d, code, _stream(stream))
     _check(rc, "favor_orf_omega_seeded")

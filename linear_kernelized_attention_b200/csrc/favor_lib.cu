@@ -330,19 +330,26 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 namespace {
 
-// Device address of the static scratch on the current device, looked up once per device.
-int noalloc_scratch(void** p) {
+// Device address of the static scratch on the current device. The address belongs to the
+// device's current context, which a device reset replaces, so it is looked up again on every
+// call that is not being captured into a graph. A call under stream capture cannot make that
+// runtime call; it takes the address the last uncaptured call on the device found.
+int noalloc_scratch(void** p, cudaStream_t st) {
   static void* addr[64] = {};
   static std::mutex mu;
   *p = nullptr;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FAVOR_ERR_CUDA;
   if (dev < 0 || dev >= 64) return FAVOR_ERR_UNSUPPORTED;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return FAVOR_ERR_CUDA;
   std::lock_guard<std::mutex> g(mu);
-  if (!addr[dev]) {
+  if (cs == cudaStreamCaptureStatusNone) {
     void* a = nullptr;
     if (cudaGetSymbolAddress(&a, favor::g_noalloc_scratch) != cudaSuccess || !a) return FAVOR_ERR_CUDA;
     addr[dev] = a;
+  } else if (!addr[dev]) {
+    return FAVOR_ERR_UNSUPPORTED;  // the first call on a device must not be captured
   }
   *p = addr[dev];
   return FAVOR_OK;
@@ -358,7 +365,7 @@ int launch_f32_static(const float* q, const float* k, const float* v, const floa
   if (BH > 65535 || nch > 65535) return FAVOR_ERR_UNSUPPORTED;
   if (f32_workspace(BH, L, d, M, kind) > favor::kNoAllocScratchBytes) return FAVOR_ERR_UNSUPPORTED;
   void* ws = nullptr;
-  int rc = noalloc_scratch(&ws);
+  int rc = noalloc_scratch(&ws, st);
   if (rc != FAVOR_OK) return rc;
   float* dS = static_cast<float*>(ws);
   float* cmax = dS + (size_t)BH * nch * F * (d + 1);
