@@ -16,6 +16,8 @@
 #include "kernels_f32.cuh"
 #include "kernel_bidir.cuh"
 #include "kernel_causal.cuh"
+#include "kernel_bidir_split.cuh"
+#include "kernel_causal_fs.cuh"
 #include "kernel_decode.cuh"
 #include "kernels_bwd_f32.cuh"
 
@@ -133,6 +135,21 @@ bool make_map_rows64(CUtensorMap* m, const void* ptr, uint64_t n1, uint64_t n2) 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 tensor [n2][n1][d] (d = 16, 32, 64 or 128 elements per row) read in boxes of
+// {64, 128, 1} with 128-byte swizzle. Columns past d and rows past n1 read as zero and are not
+// written; a row of d = 128 takes two boxes (columns 0 and 64).
+bool make_map_rows(CUtensorMap* m, const void* ptr, int d, uint64_t n1, uint64_t n2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, n1, n2};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * n1};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ scratch
 // Scratch comes from a library-owned stream-ordered pool (per device) that keeps its memory
 // between calls, so repeated calls do not return memory to the driver.
@@ -181,12 +198,139 @@ BidirPlan plan_bidir(int BH, int L, int M) {
   return pl;
 }
 
-int check_tc_shape(int d, int M, int kind) {
-  if (d != 64) return FAVOR_ERR_UNSUPPORTED;
-  if (M % 16 != 0) return FAVOR_ERR_UNSUPPORTED;
+int check_tc_shape(int d, int M, int kind, int causal) {
+  if (d != 16 && d != 32 && d != 64 && d != 128) return FAVOR_ERR_UNSUPPORTED;
   if (kind == FAVOR_TRIG && M > 256) return FAVOR_ERR_UNSUPPORTED;
   if (kind == FAVOR_RELU && M > 512) return FAVOR_ERR_UNSUPPORTED;
+  if (causal && d > 64) return FAVOR_ERR_UNSUPPORTED;
   return FAVOR_OK;
+}
+
+// ------------------------------------------------------------------ bf16 bidirectional, split
+// Shapes of the three-launch bidirectional path: key states over (pair, tile) units, the merge,
+// and queries over (head, tile) units. Every CTA takes a contiguous run of units; the grids are
+// the SM count (one CTA per SM) or the unit count if smaller.
+struct SplitPlan {
+  int dp, nab, ntiles, smax, Pk, Pq;
+  long long units_k, units_q, npairs;
+  size_t part_bytes, meta_bytes, img_bytes_head, ws_bytes;
+  int q_off_img, q_off_q, q_off_out, q_off_misc, q_smem, k_smem;
+};
+
+template <int KIND, int DP>
+void plan_split_t(SplitPlan& pl, int BH, int L, int M) {
+  using SC = bs::StateCfg<KIND, DP>;
+  using QC = bs::QueryCfg<KIND, DP>;
+  pl.dp = DP;
+  pl.nab = (M + 127) / 128;
+  pl.ntiles = (L + bs::kTile - 1) / bs::kTile;
+  pl.npairs = (long long)BH * pl.nab;
+  pl.units_k = pl.npairs * pl.ntiles;
+  pl.units_q = (long long)BH * pl.ntiles;
+  const int sms = sm_count();
+  pl.Pk = (int)std::min<long long>(sms, pl.units_k);
+  pl.Pq = (int)std::min<long long>(sms, pl.units_q);
+  const long long per = pl.units_k / pl.Pk;  // >= 1
+  pl.smax = (int)std::min<long long>(pl.Pk, (pl.ntiles + per - 1) / per + 1);
+  pl.part_bytes = (size_t)pl.npairs * pl.smax * (DP + 1) * SC::R * sizeof(float);
+  pl.meta_bytes = ((size_t)pl.npairs * pl.smax * 2 * sizeof(float) + 255) / 256 * 256;
+  pl.img_bytes_head = (size_t)pl.nab * (QC::FB / 64) * QC::NV * bs::kRowB;
+  pl.ws_bytes = pl.part_bytes + pl.meta_bytes + (size_t)BH * pl.img_bytes_head;
+  const int om_bytes = pl.nab * QC::NCB * bs::kBoxB;
+  pl.q_off_img = om_bytes;
+  pl.q_off_q = (int)((pl.q_off_img + pl.img_bytes_head + 1023) / 1024 * 1024);
+  pl.q_off_out = pl.q_off_q + 2 * QC::NCB * bs::kBoxB;
+  pl.q_off_misc = pl.q_off_out + QC::NOS * QC::NCB * bs::kBoxB;
+  pl.q_smem = pl.q_off_misc + 1024 + 1024;
+  pl.k_smem = SC::kSmem;
+}
+
+bool plan_split(SplitPlan& pl, int BH, int L, int d, int M, int kind) {
+  const int dp = d <= 64 ? 64 : 128;
+  if (kind == FAVOR_TRIG) {
+    if (dp == 64) plan_split_t<0, 64>(pl, BH, L, M); else plan_split_t<0, 128>(pl, BH, L, M);
+  } else {
+    if (dp == 64) plan_split_t<1, 64>(pl, BH, L, M); else plan_split_t<1, 128>(pl, BH, L, M);
+  }
+  return pl.q_smem <= 232448;
+}
+
+template <int KIND, int DP>
+int launch_split_t(const SplitPlan& pl, const void* q, const void* k, const void* v, const void* omega, void* out,
+                   int BH, int H, int L, int d, int M, void* ws, cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mo, mom;
+  if (!make_map_rows(&mq, q, d, L, BH) || !make_map_rows(&mk, k, d, L, BH) || !make_map_rows(&mv, v, d, L, BH) ||
+      !make_map_rows(&mo, out, d, L, BH) || !make_map_rows(&mom, omega, d, M, H))
+    return FAVOR_ERR_CUDA;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  float* part = reinterpret_cast<float*>(w8);
+  float* meta = reinterpret_cast<float*>(w8 + pl.part_bytes);
+  uint8_t* img = w8 + pl.part_bytes + pl.meta_bytes;
+
+  bs::StateParams sp{};
+  sp.H = H;
+  sp.L = L;
+  sp.M = M;
+  sp.nab = pl.nab;
+  sp.ntiles = pl.ntiles;
+  sp.units = pl.units_k;
+  sp.smax = pl.smax;
+  sp.part = part;
+  sp.meta = meta;
+  auto ks = bs::k_bidir_state<KIND, DP>;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(ks), pl.k_smem) != FAVOR_OK) return FAVOR_ERR_CUDA;
+  ks<<<pl.Pk, bs::kThreads, pl.k_smem, st>>>(mk, mv, mom, sp);
+
+  bs::MergeParams mp{};
+  mp.nab = pl.nab;
+  mp.ntiles = pl.ntiles;
+  mp.smax = pl.smax;
+  mp.M = M;
+  mp.units = pl.units_k;
+  mp.P = pl.Pk;
+  mp.part = part;
+  mp.meta = meta;
+  mp.img = img;
+  mp.img_bytes = (long long)pl.img_bytes_head;
+  bs::k_bidir_merge<KIND, DP><<<dim3((unsigned)pl.npairs, bs::StateCfg<KIND, DP>::R / 32), 256, 0, st>>>(mp);
+
+  bs::QueryParams qp{};
+  qp.H = H;
+  qp.L = L;
+  qp.M = M;
+  qp.nab = pl.nab;
+  qp.ntiles = pl.ntiles;
+  qp.units = pl.units_q;
+  qp.img = img;
+  qp.img_bytes = (int)pl.img_bytes_head;
+  qp.om_bytes = pl.nab * bs::QueryCfg<KIND, DP>::NCB * bs::kBoxB;
+  qp.off_img = pl.q_off_img;
+  qp.off_q = pl.q_off_q;
+  qp.off_out = pl.q_off_out;
+  qp.off_misc = pl.q_off_misc;
+  auto kq = bs::k_bidir_query<KIND, DP>;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(kq), pl.q_smem) != FAVOR_OK) return FAVOR_ERR_CUDA;
+  kq<<<pl.Pq, bs::kThreads, pl.q_smem, st>>>(mq, mom, mo, qp);
+  return cudaGetLastError() == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
+}
+
+int launch_bidir_split(const void* q, const void* k, const void* v, const void* omega, void* out, int B, int H,
+                       int L, int d, int M, int kind, cudaStream_t st) {
+  const int BH = B * H;
+  SplitPlan pl{};
+  if (!plan_split(pl, BH, L, d, M, kind)) return FAVOR_ERR_UNSUPPORTED;
+  if (pl.npairs > INT_MAX) return FAVOR_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  int rc = scratch_alloc(&ws, pl.ws_bytes, st);
+  if (rc != FAVOR_OK) return rc;
+  if (kind == FAVOR_TRIG)
+    rc = pl.dp == 64 ? launch_split_t<0, 64>(pl, q, k, v, omega, out, BH, H, L, d, M, ws, st)
+                     : launch_split_t<0, 128>(pl, q, k, v, omega, out, BH, H, L, d, M, ws, st);
+  else
+    rc = pl.dp == 64 ? launch_split_t<1, 64>(pl, q, k, v, omega, out, BH, H, L, d, M, ws, st)
+                     : launch_split_t<1, 128>(pl, q, k, v, omega, out, BH, H, L, d, M, ws, st);
+  cudaFreeAsync(ws, st);
+  return rc;
 }
 
 int launch_bidir_bf16(const void* q, const void* k, const void* v, const void* omega, void* out,
@@ -264,6 +408,47 @@ int launch_causal_bf16(const void* q, const void* k, const void* v, const void* 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(BH * G, 1, 1);
   cfg.blockDim = dim3(tc::kThreadsC, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = G;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mom, prm, static_cast<__nv_bfloat16*>(out)) == cudaSuccess
+             ? FAVOR_OK
+             : FAVOR_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ bf16 causal, feature split
+// One cluster of G CTAs per head, each owning 64 angles: G = ceil(M / 64) (<= 4 trig, <= 8 ReLU).
+int launch_causal_fs(const void* q, const void* k, const void* v, const void* omega, void* out, int B, int H,
+                     int L, int d, int M, int kind, cudaStream_t st) {
+  const int BH = B * H;
+  const int G0 = (M + 63) / 64;
+  const int G = G0 <= 1 ? 1 : G0 <= 2 ? 2 : G0 <= 4 ? 4 : 8;
+  if (G0 > 8 || (kind == FAVOR_TRIG && G0 > 4)) return FAVOR_ERR_UNSUPPORTED;
+  if ((long long)BH * G > INT_MAX) return FAVOR_ERR_UNSUPPORTED;
+  CUtensorMap mq, mk, mv, mom;
+  if (!make_map_rows(&mq, q, d, L, BH) || !make_map_rows(&mk, k, d, L, BH) || !make_map_rows(&mv, v, d, L, BH) ||
+      !make_map_rows(&mom, omega, d, M, H))
+    return FAVOR_ERR_CUDA;
+  cf::CausalParams prm{};
+  prm.BH = BH;
+  prm.H = H;
+  prm.L = L;
+  prm.M = M;
+  prm.G = G;
+  prm.nch = (L + cf::kTile - 1) / cf::kTile;
+  prm.d = d;
+  const uint32_t smem = cf::causal_smem_bytes();
+  auto kern = kind == FAVOR_TRIG ? cf::k_causal_fs<0> : cf::k_causal_fs<1>;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)smem) != FAVOR_OK) return FAVOR_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(BH * G, 1, 1);
+  cfg.blockDim = dim3(cf::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -518,13 +703,13 @@ int favor_attention_chunked(const void* q, const void* k, const void* v, const v
   int rc = check_common(q, k, v, omega, out, B, H, L, d, M, feature_kind);
   if (rc != FAVOR_OK) return rc;
   if ((rc = check_device()) != FAVOR_OK) return rc;
-  if ((rc = check_tc_shape(d, M, feature_kind)) != FAVOR_OK) return rc;
+  if ((rc = check_tc_shape(d, M, feature_kind, causal)) != FAVOR_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (causal) {
     if (chunk != 0 && chunk != tc::kTile) return FAVOR_ERR_UNSUPPORTED;
-    return launch_causal_bf16(q, k, v, omega, out, B, H, L, M, feature_kind, st);
+    return launch_causal_fs(q, k, v, omega, out, B, H, L, d, M, feature_kind, st);
   }
-  return launch_bidir_bf16(q, k, v, omega, out, B, H, L, M, feature_kind, st);
+  return launch_bidir_split(q, k, v, omega, out, B, H, L, d, M, feature_kind, st);
 }
 
 int favor_attention(const void* q, const void* k, const void* v, const void* omega, void* out,

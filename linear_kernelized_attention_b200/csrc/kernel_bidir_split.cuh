@@ -1,0 +1,827 @@
+// kernel_bidir_split.cuh - bidirectional FAVOR forward on sm_100a tensor cores, as three
+// launches that spread the work over every SM.
+//
+// What it computes. The explainer page "用随机特征“骗”过 softmax，Transformer 注意力也能跑成线性？",
+// section 核心机制：FAVOR+: out = D_hat^-1 phi(Q) (phi(K)^T [V|1]). The state S = phi(K)^T [V|1]
+// is aggregated first and then left-multiplied by phi(Q); no L x L matrix is formed.
+//
+// 1. k_bidir_state: key-side partial states. The work is the list of units (pair, tile) with
+//    pair = (head, 128-angle block) and tile = 128 keys, cut into one contiguous run per CTA
+//    (one CTA per SM), so every SM gets the same number of tiles whatever B*H is. Per 64-key
+//    item of a tile:
+//      MMA1  U^T = Omega_a K_item^T    (M = 128 angles, N = 64 keys, K = head dim; bf16 -> fp32 TMEM)
+//      epilogue: cos/sin (trig) or max(., 0) (ReLU) of U^T -> bf16, in place in TMEM
+//      MMA2  S_blk += phi^T [w o V | w]  (A = phi^T from TMEM, B = the V tile plus a column
+//            buffer, MN-major; M = 128 feature rows, N = d_pad + 16, K = 16 keys per instruction)
+//    Trig keys carry w_j = exp(|k_j|^2/2 - c), the exp(|x|^2/2) factor of the trig map with a
+//    running reference c kept 16 nats above the largest |k|^2/2 seen in the run; four warps
+//    compute the norms and fold w_j into row j of the V tile. When c grows, S is rescaled in
+//    TMEM first. At the end of a run of tiles of one pair, S (fp32) and (c, max |S|) go to a
+//    workspace slot.
+// 2. k_bidir_merge: per pair and 32 state rows, the slots are summed at the head's largest
+//    reference and rounded to the query-side operand type: fp16 under a power-of-two scale
+//    taken from the slots' bounds (trig), or bf16 (ReLU). The result is written in the
+//    swizzled K-major layout the query kernel's MMA reads, so one bulk copy places it.
+// 3. k_bidir_query: units (head, tile) cut into one run per CTA. Per 128-angle block of a
+//    128-query tile:
+//      MMA1  U = Q_tile Omega_ab^T      (M = 128 queries, N = 128 angles)
+//      epilogue: cos/sin or max(., 0) -> fp16/bf16 in place in TMEM (the exp(|q|^2/2) and
+//            1/sqrt(M) factors cancel between numerator and denominator)
+//      MMA2  num += phi_ab S_ab          (A from TMEM, B = the state image; N = d_pad + 16)
+//    then out = num[:, :d] / num[:, d_pad] -> bf16 -> swizzled staging -> TMA store.
+//
+// Head sizes d = 16, 32, 64 are carried in 64-column boxes (the TMA box reads zeros past d and
+// the output store clips them); d = 128 uses two boxes.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+#include "sincos_poly.cuh"
+
+namespace favor {
+namespace bs {
+
+constexpr int kTile = 128;          // tokens per tile
+constexpr int kRowB = 128;          // one 64-element 16-bit row
+constexpr int kBoxB = 128 * kRowB;  // one TMA box: 128 rows x 64 elements
+constexpr float kMargin = 16.f;     // stabiliser head-room above the largest |k|^2/2 seen (nats)
+constexpr int kThreads = 512;
+
+// Angles of 8 consecutive ones evaluated on the FMA pipe (bit j set: angle j of the group);
+// the rest go to the SFU. 0x49 = 3 of 8.
+#ifndef FAVOR_POLY_MASK
+#define FAVOR_POLY_MASK 0x49u
+#endif
+constexpr uint32_t kPolyMask = FAVOR_POLY_MASK;
+
+// Contiguous runs of units: CTA i owns units [floor(i U / P), floor((i + 1) U / P)).
+__host__ __device__ inline long long run_begin(long long i, long long U, long long P) { return i * U / P; }
+__host__ __device__ inline long long cta_of_unit(long long x, long long U, long long P) {
+  return ((x + 1) * P - 1) / U;
+}
+
+// ============================================================================ key states
+template <int KIND, int DP>
+struct StateCfg {
+  static constexpr int NCB = DP / 64;                        // 64-column boxes of a row
+  static constexpr int NV = DP + 16;                         // MMA2 N: values, normaliser (column DP), pad
+  static constexpr int NSB = KIND == 0 ? 2 : 1;              // 128-row state blocks (trig: cos, sin)
+  static constexpr int R = 128 * NSB;                        // state rows of a pair
+  static constexpr int NBUF = (KIND == 0 && DP == 128) ? 3 : 4;  // 64-key U/phi buffers
+  static constexpr int NS = DP == 64 ? 3 : 2;                // K/V stages
+  static constexpr int kStageB = (2 * NCB + 1) * kBoxB;      // V boxes | column box | K boxes
+  static constexpr int kOmB = NCB * kBoxB;                   // one Omega block
+  static constexpr int kUcol = (NSB * NV + 31) / 32 * 32;    // TMEM column of the U ring
+  static constexpr int kMiscOff = 2 * kOmB + NS * kStageB;
+  static constexpr int kSmem = kMiscOff + 1024 + 1024;       // misc block + alignment slack
+  static_assert(kUcol + NBUF * 64 <= 512, "TMEM budget");
+  static_assert(kSmem <= 232448, "shared memory budget");
+};
+
+struct StateParams {
+  int H, L, M;
+  int nab;        // 128-angle blocks
+  int ntiles;     // 128-key tiles per head
+  long long units;  // B * H * nab * ntiles
+  int smax;       // workspace slots per pair
+  float* part;    // [pair * smax + slot][d_pad + 1][R] fp32
+  float* meta;    // [pair * smax + slot][2]: reference c (trig), max |entry|
+};
+
+struct alignas(16) StateMisc {
+  int abort_flag;
+  uint32_t tmem_base;
+  float tmax[2][4];
+  float frescale[4];
+  float redmax[2][8];
+  uint64_t om_full[2], om_free[2];
+  uint64_t kv_full[3], kv_empty[3], w_full[3];
+  uint64_t u_full[4], p_full[4], buf_free[4];
+  uint64_t s_done, s_free, drain;
+  uint64_t norm_sync;  // bounded barrier among the 128 norm threads
+};
+static_assert(sizeof(StateMisc) <= 1024, "misc block");
+
+template <int KIND, int DP>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_bidir_state(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_om, const StateParams p) {
+  using C = StateCfg<KIND, DP>;
+  constexpr int NCB = C::NCB, NV = C::NV, NSB = C::NSB, R = C::R, NBUF = C::NBUF, NS = C::NS;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gb = smem_raw + (base - raw);
+  const uint32_t s_om = base, s_stage = base + 2 * C::kOmB;
+  StateMisc* ms = reinterpret_cast<StateMisc*>(gb + C::kMiscOff);
+  volatile int* abort_flag = &ms->abort_flag;
+  auto bar = [](uint64_t& b) { return smem_u32(&b); };
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long P = gridDim.x, U = p.units;
+  const long long u0 = run_begin(blockIdx.x, U, P), u1 = run_begin(blockIdx.x + 1, U, P);
+  const int n = (int)(u1 - u0);  // tiles of this CTA
+  const int nt = p.ntiles;
+  const long long p0 = u0 / nt;  // first pair of the run
+  auto pair_of = [&](int t) { return (u0 + t) / nt; };
+  auto first_of_pair = [&](int t) { return t == 0 || (u0 + t) % nt == 0; };
+  auto last_of_pair = [&](int t) { return t == n - 1 || (u0 + t) % nt == nt - 1; };
+  auto slot_of = [&](long long pr) {
+    return pr * p.smax + (blockIdx.x - cta_of_unit(pr * nt, U, P));
+  };
+
+  // ---------------------------------------------------------------- set-up
+  if (tid == 0) {
+    ms->abort_flag = 0;
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(ms->om_full[i]), 1);
+      mbar_init(bar(ms->om_free[i]), 1);
+    }
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar(ms->kv_full[s]), 1);
+      mbar_init(bar(ms->kv_empty[s]), 1);
+      mbar_init(bar(ms->w_full[s]), 4);
+    }
+    for (int b = 0; b < NBUF; ++b) {
+      mbar_init(bar(ms->u_full[b]), 1);
+      mbar_init(bar(ms->p_full[b]), 4);
+      mbar_init(bar(ms->buf_free[b]), 1);
+    }
+    mbar_init(bar(ms->s_done), 1);
+    mbar_init(bar(ms->s_free), 8);
+    mbar_init(bar(ms->drain), 1);
+    mbar_init(bar(ms->norm_sync), 128);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ms->tmem_base), 512);
+    tmem_relinquish();
+  }
+  {  // column boxes: zero, with the normaliser column (element 0 of each row) 1.0 for ReLU
+    for (int s = 0; s < NS; ++s) {
+      uint4* col = reinterpret_cast<uint4*>(gb + (s_stage - base) + s * C::kStageB + NCB * kBoxB);
+      for (int i = tid; i < kBoxB / 16; i += kThreads) col[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncthreads();
+    if (KIND == 1 && tid < kTile)
+      for (int s = 0; s < NS; ++s)
+        *reinterpret_cast<uint16_t*>(gb + (s_stage - base) + s * C::kStageB + NCB * kBoxB + tid * kRowB +
+                                     ((tid & 7) << 4)) = 0x3F80u;
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && n > 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_om);
+      int issued = 0, pk_issued = 0;
+      for (int t = 0; t < n; ++t) {
+        const long long x = u0 + t, pr = x / nt;
+        const int pk = (int)(pr - p0);
+        const int bh = (int)(pr / p.nab), ab = (int)(pr % p.nab), h = bh % p.H;
+        if (first_of_pair(t)) {
+          if (pk >= 2 && !mbar_wait(bar(ms->om_free[pk & 1]), ((pk >> 1) - 1) & 1, abort_flag)) break;
+          mbar_arrive_expect_tx(bar(ms->om_full[pk & 1]), C::kOmB);
+          for (int kb = 0; kb < NCB; ++kb)
+            tma_load_3d(s_om + (pk & 1) * C::kOmB + kb * kBoxB, &tm_om, bar(ms->om_full[pk & 1]), kb * 64, ab * 128, h);
+          pk_issued = pk + 1;
+        }
+        const int s = t % NS;
+        if (t >= NS && !mbar_wait(bar(ms->kv_empty[s]), ((t / NS) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(ms->kv_full[s]), 2 * NCB * kBoxB);
+        const uint32_t st = s_stage + s * C::kStageB;
+        const int row = (int)(x % nt) * kTile;
+        for (int kb = 0; kb < NCB; ++kb) {
+          tma_load_3d(st + kb * kBoxB, &tm_v, bar(ms->kv_full[s]), kb * 64, row, bh);
+          tma_load_3d(st + (NCB + 1 + kb) * kBoxB, &tm_k, bar(ms->kv_full[s]), kb * 64, row, bh);
+        }
+        issued = t + 1;
+      }
+      if (*abort_flag) {  // let the copies already issued land before the CTA can exit
+        constexpr long long kDrain = kWaitLimitCycles / 8;
+        for (int t = issued > NS ? issued - NS : 0; t < issued; ++t)
+          mbar_wait(bar(ms->kv_full[t % NS]), (t / NS) & 1, nullptr, kDrain);
+        for (int pk = pk_issued > 2 ? pk_issued - 2 : 0; pk < pk_issued; ++pk)
+          mbar_wait(bar(ms->om_full[pk & 1]), (pk >> 1) & 1, nullptr, kDrain);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n > 0) {
+      const uint32_t id1 = idesc_f16(128, 64, 1, 1, 0, 0);
+      const uint32_t id2 = idesc_f16(128, NV, 1, 1, 0, 1);
+      const int nitems = 2 * n;
+      bool ok = true;
+      auto mma1 = [&](int it) -> bool {
+        const int t = it >> 1, hf = it & 1, s = t % NS, b = it % NBUF;
+        const int pk = (int)(pair_of(t) - p0);
+        if (hf == 0) {
+          if (first_of_pair(t) && !mbar_wait(bar(ms->om_full[pk & 1]), (pk >> 1) & 1, abort_flag)) return false;
+          if (!mbar_wait(bar(ms->kv_full[s]), (t / NS) & 1, abort_flag)) return false;
+        }
+        tc_fence_after();
+        const uint64_t a0 = sdesc_sw128(s_om + (pk & 1) * C::kOmB, 16, 1024);
+        const uint64_t b0 = sdesc_sw128(s_stage + s * C::kStageB + (NCB + 1) * kBoxB + hf * 64 * kRowB, 16, 1024);
+        const uint32_t d = tmem + C::kUcol + b * 64;
+#pragma unroll
+        for (int kb = 0; kb < NCB; ++kb)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t off = uint64_t((kb * kBoxB + kk * 32) >> 4);
+            mma_ss(d, a0 + off, b0 + off, id1, (kb | kk) ? 1u : 0u);
+          }
+        mma_commit(bar(ms->u_full[b]));
+        if (hf == 1 && last_of_pair(t)) mma_commit(bar(ms->om_free[pk & 1]));
+        return true;
+      };
+      auto write_meta_max = [&](int pk) {
+        float mx = 0.f;
+        for (int w = 0; w < 8; ++w) mx = fmaxf(mx, ms->redmax[pk & 1][w]);
+        const long long sl = slot_of(p0 + pk);
+        p.meta[sl * 2 + 1] = mx;
+        if (KIND == 1) p.meta[sl * 2] = 0.f;
+      };
+      for (int it = 0; ok && it < NBUF && it < nitems; ++it) ok = mma1(it);
+      for (int it = 0; ok && it < nitems; ++it) {
+        const int t = it >> 1, hf = it & 1, s = t % NS, b = it % NBUF;
+        const int pk = (int)(pair_of(t) - p0);
+        const bool fresh = hf == 0 && first_of_pair(t);
+        if (!(ok = mbar_wait(bar(ms->p_full[b]), (it / NBUF) & 1, abort_flag))) break;
+        if (KIND == 0 && hf == 0 && !(ok = mbar_wait(bar(ms->w_full[s]), (t / NS) & 1, abort_flag))) break;
+        if (fresh && pk > 0) {
+          if (!(ok = mbar_wait(bar(ms->s_free), (pk - 1) & 1, abort_flag))) break;
+          write_meta_max(pk - 1);
+        }
+        tc_fence_after();
+        const uint64_t vd =
+            sdesc_sw128(s_stage + s * C::kStageB, kBoxB, 1024) + uint64_t((hf * 64 * kRowB) >> 4);
+        const uint32_t ub = tmem + C::kUcol + b * 64;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bd = vd + uint64_t((kk * 16 * kRowB) >> 4);
+          const uint32_t acc = (fresh && kk == 0) ? 0u : 1u;
+          const uint32_t col = 32 * (kk >> 1) + 8 * (kk & 1);
+          mma_ts(tmem, ub + col, bd, id2, acc);
+          if (KIND == 0) mma_ts(tmem + NV, ub + 16 + col, bd, id2, acc);
+        }
+        mma_commit(bar(ms->buf_free[b]));
+        if (hf == 1) {
+          mma_commit(bar(ms->kv_empty[s]));
+          if (last_of_pair(t)) mma_commit(bar(ms->s_done));
+        }
+        const int nx = it + NBUF;
+        if (nx < nitems) {
+          if (!(ok = mbar_wait(bar(ms->buf_free[b]), (it / NBUF) & 1, abort_flag))) break;
+          if (!(ok = mma1(nx))) break;
+        }
+      }
+      if (ok) {
+        const int pk_last = (int)(pair_of(n - 1) - p0);
+        if (mbar_wait(bar(ms->s_free), pk_last & 1, abort_flag)) write_meta_max(pk_last);
+      }
+      mma_commit(bar(ms->drain));
+      mbar_wait(bar(ms->drain), 0, nullptr, kWaitLimitCycles / 8);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ key norms (trig)
+    if (KIND == 0 && n > 0) {
+      const int j = (warp - 4) * 32 + lane;  // key row of the tile
+      float c = 0.f;
+      uint32_t nph = 0;
+      for (int t = 0; t < n; ++t) {
+        const long long x = u0 + t;
+        const int s = t % NS;
+        if (!mbar_wait(bar(ms->kv_full[s]), (t / NS) & 1, abort_flag)) break;
+        uint8_t* st = gb + (s_stage - base) + s * C::kStageB;
+        float acc = 0.f;
+#pragma unroll
+        for (int kb = 0; kb < NCB; ++kb)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint4 xv =
+                *reinterpret_cast<const uint4*>(st + (NCB + 1 + kb) * kBoxB + j * kRowB + ((ch ^ (j & 7)) << 4));
+            const uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float lo = __uint_as_float(w4[e] << 16), hi = __uint_as_float(w4[e] & 0xFFFF0000u);
+              acc = fmaf(lo, lo, acc);
+              acc = fmaf(hi, hi, acc);
+            }
+          }
+        const bool valid = (int)(x % nt) * kTile + j < p.L;
+        const float n2 = valid ? 0.5f * acc : -INFINITY;
+        float m = n2;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) ms->tmax[t & 1][warp - 4] = m;
+        if (!group_sync(bar(ms->norm_sync), nph, abort_flag)) break;
+        m = fmaxf(fmaxf(ms->tmax[t & 1][0], ms->tmax[t & 1][1]), fmaxf(ms->tmax[t & 1][2], ms->tmax[t & 1][3]));
+        float f = 1.f;
+        if (first_of_pair(t)) {
+          c = m + kMargin;
+        } else if (m > c) {
+          const float cn = m + kMargin;
+          f = __expf(c - cn);
+          c = cn;
+        }
+        const float w = valid ? __expf(n2 - c) : 0.f;
+#pragma unroll
+        for (int kb = 0; kb < NCB; ++kb)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            uint4* px = reinterpret_cast<uint4*>(st + kb * kBoxB + j * kRowB + ((ch ^ (j & 7)) << 4));
+            const uint4 xv = *px;
+            const uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};
+            uint32_t o4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              o4[e] = pack_bf16x2(__uint_as_float(w4[e] << 16) * w, __uint_as_float(w4[e] & 0xFFFF0000u) * w);
+            *px = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+          }
+        *reinterpret_cast<__nv_bfloat16*>(st + NCB * kBoxB + j * kRowB + ((j & 7) << 4)) = __float2bfloat16_rn(w);
+        if (j == 0) {
+          ms->frescale[s] = f;
+          if (last_of_pair(t)) p.meta[slot_of(x / nt) * 2] = c;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(ms->w_full[s]));
+      }
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ features and state flushes
+    const int g = (warp - 8) >> 2, q = warp & 3;
+    const uint32_t la = uint32_t(q * 32) << 16;
+    const int nitems = 2 * n;
+    bool ok = true;
+    for (int it = g; ok && it < nitems; it += 2) {
+      const int t = it >> 1, hf = it & 1, s = t % NS, b = it % NBUF;
+      if (!(ok = mbar_wait(bar(ms->u_full[b]), (it / NBUF) & 1, abort_flag))) break;
+      if (KIND == 0 && hf == 0 && !first_of_pair(t)) {
+        // the tile raised the reference: rescale S once every earlier state MMA has completed
+        if (!(ok = mbar_wait(bar(ms->w_full[s]), (t / NS) & 1, abort_flag))) break;
+        const float f = ms->frescale[s];
+        if (f != 1.f) {
+          if (!(ok = mbar_wait(bar(ms->buf_free[(it - 1) % NBUF]), ((it - 1) / NBUF) & 1, abort_flag))) break;
+          tc_fence_after();
+          for (int c0 = 0; c0 < NSB * NV; c0 += 8) {
+            uint32_t r8[8];
+            tmem_ld8(tmem + la + c0, r8);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 8; ++e) r8[e] = __float_as_uint(__uint_as_float(r8[e]) * f);
+            tmem_st8(tmem + la + c0, r8);
+          }
+          tmem_wait_st();
+        }
+      }
+      tc_fence_after();
+      const uint32_t ub = tmem + la + C::kUcol + b * 64;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t u[32];
+        tmem_ld32(ub + 32 * c, u);
+        tmem_wait_ld();
+        if (KIND == 0) {
+          uint32_t cp[16], sp[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float s0, c0, s1, c1;
+            sincos_mixed<kPolyMask>(2 * e, __uint_as_float(u[2 * e]), s0, c0);
+            sincos_mixed<kPolyMask>(2 * e + 1, __uint_as_float(u[2 * e + 1]), s1, c1);
+            cp[e] = pack_bf16x2(c0, c1);
+            sp[e] = pack_bf16x2(s0, s1);
+          }
+          tmem_st16(ub + 32 * c, cp);
+          tmem_st16(ub + 32 * c + 16, sp);
+        } else {
+          uint32_t rp[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            rp[e] = pack_bf16x2(fmaxf(__uint_as_float(u[2 * e]), 0.f), fmaxf(__uint_as_float(u[2 * e + 1]), 0.f));
+          tmem_st16(ub + 32 * c, rp);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(ms->p_full[b]));
+      if (last_of_pair(t)) {
+        // flush: this group's share of the state to the pair's workspace slot
+        const long long pr = pair_of(t);
+        const int pk = (int)(pr - p0);
+        if (!(ok = mbar_wait(bar(ms->s_done), pk & 1, abort_flag))) break;
+        tc_fence_after();
+        float* dst = p.part + slot_of(pr) * (long long)(DP + 1) * R;
+        float mx = 0.f;
+        // trig: group g writes state block g (rows g*128 ..); ReLU: group g writes value
+        // columns [g*DP/2, (g+1)*DP/2) and group 1 the normaliser column
+        const int row = (KIND == 0 ? g * 128 : 0) + q * 32 + lane;
+        const uint32_t sa = tmem + la + (KIND == 0 ? g * NV : 0);
+        const int c_lo = KIND == 0 ? 0 : g * (DP / 2), c_hi = KIND == 0 ? DP : (g + 1) * (DP / 2);
+#pragma unroll 1
+        for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(sa + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float x = __uint_as_float(v[e]);
+            dst[(long long)(c0 + e) * R + row] = x;
+            mx = fmaxf(mx, fabsf(x));
+          }
+        }
+        if (KIND == 0 || g == 1) {
+          uint32_t zc;
+          tmem_ld1(sa + DP, zc);
+          tmem_wait_ld();
+          const float x = __uint_as_float(zc);
+          dst[(long long)DP * R + row] = x;
+          mx = fmaxf(mx, fabsf(x));
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) ms->redmax[pk & 1][warp - 8] = mx;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(ms->s_free));
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ============================================================================ merge
+struct MergeParams {
+  int nab, ntiles, smax, M;
+  long long units, P;   // the state kernel's unit count and grid size
+  const float* part;
+  const float* meta;
+  uint8_t* img;         // [B*H][image bytes]
+  long long img_bytes;  // per head
+};
+
+__device__ __forceinline__ int nslots(long long pr, const MergeParams& p) {
+  return (int)(cta_of_unit((pr + 1) * p.ntiles - 1, p.units, p.P) - cta_of_unit(pr * p.ntiles, p.units, p.P) + 1);
+}
+
+// Byte of (feature f, value row n) in a K-major 128-byte-swizzled image of NV rows per
+// 64-feature atom.
+template <int NV>
+__device__ __forceinline__ uint32_t img_byte(int f, int n) {
+  return uint32_t(f >> 6) * (NV * kRowB) + uint32_t(n) * kRowB + ((uint32_t(((f & 63) >> 3) ^ (n & 7))) << 4) +
+         uint32_t(f & 7) * 2;
+}
+
+// One block per (pair, 32 state rows). Trig feature order within a 128-angle block: 32-angle
+// groups of [cos 32 | sin 32], matching the query kernel's packing.
+template <int KIND, int DP>
+__global__ void __launch_bounds__(256) k_bidir_merge(const MergeParams p) {
+  constexpr int NV = DP + 16, R = KIND == 0 ? 256 : 128, FB = R;
+  const long long pr = blockIdx.x;
+  const int rb = blockIdx.y;
+  const long long bh = pr / p.nab;
+  const int ab = (int)(pr % p.nab);
+  // the head's reference and the bound of its merged state
+  float cmax = -INFINITY;
+  for (int a2 = 0; a2 < p.nab; ++a2) {
+    const long long q2 = bh * p.nab + a2;
+    const int ns = nslots(q2, p);
+    for (int s = 0; s < ns; ++s) cmax = fmaxf(cmax, p.meta[(q2 * p.smax + s) * 2]);
+  }
+  float bound = 0.f;
+  for (int a2 = 0; a2 < p.nab; ++a2) {
+    const long long q2 = bh * p.nab + a2;
+    const int ns = nslots(q2, p);
+    for (int s = 0; s < ns; ++s) {
+      const float* m = p.meta + (q2 * p.smax + s) * 2;
+      bound += (KIND == 0 ? __expf(m[0] - cmax) : 1.f) * m[1];
+    }
+  }
+  const float scale = (KIND == 0 && bound > 0.f) ? exp2f(14.f - ceilf(log2f(bound))) : 1.f;
+  const int ns = nslots(pr, p);
+  uint8_t* img = p.img + bh * p.img_bytes;
+  for (int e = threadIdx.x; e < 32 * NV; e += blockDim.x) {
+    const int rl = e & 31, nn = e >> 5;
+    const int r = rb * 32 + rl;
+    float v = 0.f;
+    if (nn <= DP) {
+      for (int s = 0; s < ns; ++s) {
+        const long long sl = pr * p.smax + s;
+        const float w = KIND == 0 ? __expf(p.meta[sl * 2] - cmax) : 1.f;
+        v = fmaf(w, p.part[(sl * (DP + 1) + nn) * R + r], v);
+      }
+    }
+    const int a = KIND == 0 ? (r & 127) : r;
+    if (ab * 128 + a >= p.M) v = 0.f;  // padded angle
+    const int f = KIND == 0 ? ab * FB + (a >> 5) * 64 + (r >> 7) * 32 + (a & 31) : ab * FB + r;
+    if (KIND == 0)
+      *reinterpret_cast<__half*>(img + img_byte<NV>(f, nn)) = __float2half_rn(v * scale);
+    else
+      *reinterpret_cast<__nv_bfloat16*>(img + img_byte<NV>(f, nn)) = __float2bfloat16_rn(v);
+  }
+}
+
+// ============================================================================ queries
+template <int KIND, int DP>
+struct QueryCfg {
+  static constexpr int NCB = DP / 64, NV = DP + 16;
+  static constexpr int FB = KIND == 0 ? 256 : 128;   // features of a 128-angle block
+  static constexpr int NBN = DP == 64 ? 2 : 1;       // numerator buffers
+  static constexpr int NOS = DP == 64 ? 2 : 1;       // output staging buffers
+  static constexpr int kNumCol = 256;                // TMEM: U ring [0, 256), numerators after
+  static_assert(kNumCol + NBN * NV <= 512, "TMEM budget");
+};
+
+struct QueryParams {
+  int H, L, M, nab, ntiles;
+  long long units;          // B * H * ntiles
+  const uint8_t* img;       // [B*H][img_bytes]
+  int img_bytes;
+  int om_bytes;             // nab * NCB boxes
+  int off_img, off_q, off_out, off_misc;  // shared-memory layout (bytes from the aligned base)
+};
+
+struct alignas(16) QueryMisc {
+  int abort_flag;
+  uint32_t tmem_base;
+  uint64_t head_full, head_free;
+  uint64_t q_full[2], q_empty[2];
+  uint64_t u_full[2], p_full[2], buf_free[2];
+  uint64_t num_full[2], num_empty[2];
+  uint64_t drain;
+  uint64_t out_sync;  // bounded barrier among the 128 output threads
+};
+
+template <int KIND, int DP>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_bidir_query(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_om,
+                  const __grid_constant__ CUtensorMap tm_out, const QueryParams p) {
+  using C = QueryCfg<KIND, DP>;
+  constexpr int NCB = C::NCB, NV = C::NV, FB = C::FB, NBN = C::NBN, NOS = C::NOS;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gb = smem_raw + (base - raw);
+  const uint32_t s_om = base, s_img = base + p.off_img, s_q = base + p.off_q, s_out = base + p.off_out;
+  QueryMisc* ms = reinterpret_cast<QueryMisc*>(gb + p.off_misc);
+  volatile int* abort_flag = &ms->abort_flag;
+  auto bar = [](uint64_t& b) { return smem_u32(&b); };
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long P = gridDim.x, U = p.units;
+  const long long u0 = run_begin(blockIdx.x, U, P), u1 = run_begin(blockIdx.x + 1, U, P);
+  const int n = (int)(u1 - u0);
+  const int nt = p.ntiles, nab = p.nab;
+  const long long h0 = u0 / nt;
+  auto head_of = [&](int t) { return (u0 + t) / nt; };
+  auto first_of_head = [&](int t) { return t == 0 || (u0 + t) % nt == 0; };
+  auto last_of_head = [&](int t) { return t == n - 1 || (u0 + t) % nt == nt - 1; };
+
+  if (tid == 0) {
+    ms->abort_flag = 0;
+    mbar_init(bar(ms->head_full), 1);
+    mbar_init(bar(ms->head_free), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(ms->q_full[i]), 1);
+      mbar_init(bar(ms->q_empty[i]), 1);
+      mbar_init(bar(ms->u_full[i]), 1);
+      mbar_init(bar(ms->p_full[i]), 8);
+      mbar_init(bar(ms->buf_free[i]), 1);
+      mbar_init(bar(ms->num_full[i]), 1);
+      mbar_init(bar(ms->num_empty[i]), 4);
+    }
+    mbar_init(bar(ms->drain), 1);
+    mbar_init(bar(ms->out_sync), 128);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ms->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && n > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_om);
+      tma_prefetch_desc(&tm_out);
+      int issued = 0, heads = 0;
+      for (int t = 0; t < n; ++t) {
+        const long long x = u0 + t, bh = x / nt;
+        const int s = t & 1;
+        if (t >= 2 && !mbar_wait(bar(ms->q_empty[s]), ((t >> 1) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(ms->q_full[s]), NCB * kBoxB);
+        for (int kb = 0; kb < NCB; ++kb)
+          tma_load_3d(s_q + (s * NCB + kb) * kBoxB, &tm_q, bar(ms->q_full[s]), kb * 64, (int)(x % nt) * kTile, (int)bh);
+        issued = t + 1;
+        if (first_of_head(t)) {
+          const int hk = (int)(bh - h0);
+          if (hk >= 1 && !mbar_wait(bar(ms->head_free), (hk - 1) & 1, abort_flag)) break;
+          mbar_arrive_expect_tx(bar(ms->head_full), p.om_bytes + p.img_bytes);
+          const int h = (int)(bh % p.H);
+          for (int ab = 0; ab < nab; ++ab)
+            for (int kb = 0; kb < NCB; ++kb)
+              tma_load_3d(s_om + (ab * NCB + kb) * kBoxB, &tm_om, bar(ms->head_full), kb * 64, ab * 128, h);
+          const uint8_t* src = p.img + bh * p.img_bytes;
+          for (int off = 0; off < p.img_bytes; off += 32768) {
+            const int sz = min(32768, p.img_bytes - off);
+            bulk_load(s_img + off, src + off, sz, bar(ms->head_full));
+          }
+          heads = hk + 1;
+        }
+      }
+      if (*abort_flag) {
+        constexpr long long kDrain = kWaitLimitCycles / 8;
+        for (int t = issued > 2 ? issued - 2 : 0; t < issued; ++t)
+          mbar_wait(bar(ms->q_full[t & 1]), (t >> 1) & 1, nullptr, kDrain);
+        if (heads > 0) mbar_wait(bar(ms->head_full), (heads - 1) & 1, nullptr, kDrain);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n > 0) {
+      const uint32_t id1 = idesc_f16(128, 128, 1, 1, 0, 0);
+      const uint32_t fmt = KIND == 0 ? 0u : 1u;  // fp16 (trig) or bf16 (ReLU) state operands
+      const uint32_t id2 = idesc_f16(128, NV, fmt, fmt, 0, 0);
+      const int nit = n * nab;
+      const uint64_t om0 = sdesc_sw128(s_om, 16, 1024);
+      const uint64_t img0 = sdesc_sw128(s_img, 16, 1024);
+      bool ok = true;
+      auto mma1 = [&](int j) -> bool {
+        const int t = j / nab, ab = j % nab, b = j & 1, s = t & 1;
+        if (ab == 0) {
+          if (!mbar_wait(bar(ms->q_full[s]), (t >> 1) & 1, abort_flag)) return false;
+          if (first_of_head(t) && !mbar_wait(bar(ms->head_full), (int)(head_of(t) - h0) & 1, abort_flag))
+            return false;
+        }
+        if (j >= 2 && !mbar_wait(bar(ms->buf_free[b]), ((j - 2) >> 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint64_t q0 = sdesc_sw128(s_q + s * NCB * kBoxB, 16, 1024);
+#pragma unroll
+        for (int kb = 0; kb < NCB; ++kb)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + b * 128, q0 + uint64_t((kb * kBoxB + kk * 32) >> 4),
+                   om0 + uint64_t(((ab * NCB + kb) * kBoxB + kk * 32) >> 4), id1, (kb | kk) ? 1u : 0u);
+        mma_commit(bar(ms->u_full[b]));
+        if (ab == nab - 1) mma_commit(bar(ms->q_empty[s]));
+        return true;
+      };
+      int nx = 0;  // next item whose projection is to be issued
+      while (ok && nx < nit && nx < 2 && head_of(nx / nab) == h0) ok = mma1(nx++);
+      for (int j = 0; ok && j < nit; ++j) {
+        const int t = j / nab, ab = j % nab, b = j & 1, nb = t % NBN;
+        if (!(ok = mbar_wait(bar(ms->p_full[b]), (j >> 1) & 1, abort_flag))) break;
+        if (ab == 0 && t >= NBN && !(ok = mbar_wait(bar(ms->num_empty[nb]), ((t / NBN) - 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t dn = tmem + C::kNumCol + nb * NV;
+#pragma unroll
+        for (int kk = 0; kk < FB / 16; ++kk) {
+          const int f = ab * FB + 16 * kk;
+          const uint64_t bd = img0 + uint64_t(((f >> 6) * (NV * kRowB) + ((f & 63) >> 4) * 32) >> 4);
+          const uint32_t acol = KIND == 0 ? 8 * kk : 64 * (kk >> 2) + 8 * (kk & 3);
+          mma_ts(dn, tmem + b * 128 + acol, bd, id2, (ab | kk) ? 1u : 0u);
+        }
+        mma_commit(bar(ms->buf_free[b]));
+        const bool head_end = ab == nab - 1 && last_of_head(t);
+        if (ab == nab - 1) mma_commit(bar(ms->num_full[nb]));
+        if (head_end) mma_commit(bar(ms->head_free));
+        // projections ahead: two items in flight, and none past a head change until the head's
+        // last state product has been issued (the next head's Omega and image replace these)
+        while (ok && nx < nit && nx <= j + 2) {
+          const long long hn = head_of(nx / nab), hc = head_of(t);
+          if (!(hn == hc || (head_end && hn == hc + 1))) break;
+          ok = mma1(nx++);
+        }
+      }
+      mma_commit(bar(ms->drain));
+      mbar_wait(bar(ms->drain), 0, nullptr, kWaitLimitCycles / 8);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ normalise and store
+    const int q = warp & 3, row = q * 32 + lane;
+    const uint32_t la = uint32_t(q * 32) << 16;
+    const bool issuer = warp == 4 && lane == 0;
+    uint32_t oph = 0;
+    for (int t = 0; t < n; ++t) {
+      const int nb = t % NBN, sb = t % NOS;
+      if (!mbar_wait(bar(ms->num_full[nb]), (t / NBN) & 1, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t dn = tmem + la + C::kNumCol + nb * NV;
+      uint32_t dv;
+      tmem_ld1(dn + DP, dv);
+      tmem_wait_ld();
+      const float den = __uint_as_float(dv);
+      const float inv = den != 0.f ? 1.f / den : 0.f;
+      if (issuer && t >= NOS) {
+        if (NOS == 2)
+          bulk_wait_read1();
+        else
+          bulk_wait_read0();
+      }
+      if (!group_sync(bar(ms->out_sync), oph, abort_flag)) break;
+      uint8_t* stg = gb + (s_out - base) + sb * NCB * kBoxB + row * kRowB;
+#pragma unroll 1
+      for (int kb = 0; kb < NCB; ++kb) {
+        uint32_t v[32], w[32];
+        tmem_ld32(dn + kb * 64, v);
+        tmem_ld32(dn + kb * 64 + 32, w);
+        tmem_wait_ld();
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const uint32_t* src = m < 4 ? v + 8 * m : w + 8 * (m - 4);
+          *reinterpret_cast<uint4*>(stg + kb * kBoxB + ((m ^ (row & 7)) << 4)) = make_uint4(
+              pack_bf16x2(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv),
+              pack_bf16x2(__uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv),
+              pack_bf16x2(__uint_as_float(src[4]) * inv, __uint_as_float(src[5]) * inv),
+              pack_bf16x2(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(ms->num_empty[nb]));
+      fence_proxy_async_smem();
+      if (!group_sync(bar(ms->out_sync), oph, abort_flag)) break;
+      if (issuer) {
+        const long long x = u0 + t;
+        for (int kb = 0; kb < NCB; ++kb)
+          tma_store_3d(&tm_out, s_out + (sb * NCB + kb) * kBoxB, kb * 64, (int)(x % nt) * kTile, (int)(x / nt));
+        bulk_commit();
+      }
+    }
+    if (issuer) bulk_wait0();
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ query features
+    const int q = warp & 3, hcol = (warp - 8) >> 2;
+    const uint32_t la = uint32_t(q * 32) << 16;
+    const int nit = n * nab;
+    for (int j = 0; j < nit; ++j) {
+      const int b = j & 1;
+      if (!mbar_wait(bar(ms->u_full[b]), (j >> 1) & 1, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t ub = tmem + la + b * 128 + 64 * hcol;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t u[32];
+        tmem_ld32(ub + 32 * c, u);
+        tmem_wait_ld();
+        if (KIND == 0) {
+          uint32_t cp[16], sp[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float s0, c0, s1, c1;
+            sincos_mixed<kPolyMask>(2 * e, __uint_as_float(u[2 * e]), s0, c0);
+            sincos_mixed<kPolyMask>(2 * e + 1, __uint_as_float(u[2 * e + 1]), s1, c1);
+            cp[e] = pack_f16x2(c0, c1);
+            sp[e] = pack_f16x2(s0, s1);
+          }
+          tmem_st16(ub + 32 * c, cp);
+          tmem_st16(ub + 32 * c + 16, sp);
+        } else {
+          uint32_t rp[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            rp[e] = pack_bf16x2(fmaxf(__uint_as_float(u[2 * e]), 0.f), fmaxf(__uint_as_float(u[2 * e + 1]), 0.f));
+          tmem_st16(ub + 16 * c, rp);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(ms->p_full[b]));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace bs
+}  // namespace favor

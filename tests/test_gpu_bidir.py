@@ -112,3 +112,28 @@ def test_bidir_long_sequence_sampled_rows():
     ref, cond, _ = c.oracle(0, False, heads=heads, rows=rows)
     sel = np.stack([g[h][rows] for _, h in heads])
     check_rows(sel, ref, cond, TOL_BF16, U_BF16, "L=65536 sampled")
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+@pytest.mark.parametrize("d,M", [(16, 32), (32, 96), (128, 128), (16, 256), (128, 40)])
+def test_bidir_head_sizes(kind, d, M):
+    # head sizes 16 and 32 ride in the 64-column box (zeros past d, stores clipped); 128 takes two
+    # boxes. Several tiles with a ragged tail, two heads per batch entry, padded angle blocks.
+    B, H, L = 2, 2, 700
+    c = Case(B, H, L, d, M, seed=d * 7 + M)
+    g = _run(c, kind).reshape(B * H, L, d)
+    ref, cond, _ = c.oracle(kind, False)
+    check_rows(g, ref, cond, TOL_BF16, U_BF16, f"d={d} M={M} kind={kind}", trig=kind == 0)
+
+
+def test_bidir_unsupported_shapes_are_refused():
+    import torch
+    import linear_kernelized_attention_b200 as F
+    # d = 128 with trig M = 256: the state image (512 features x 144 rows) and the operand tiles do
+    # not fit in one CTA's shared memory; d = 48 is not a supported head size
+    for (d, M, kind) in ((128, 256, 0), (48, 64, 0)):
+        q = torch.zeros((1, 1, 128, d), dtype=torch.bfloat16, device="cuda")
+        om = torch.zeros((1, M, d), dtype=torch.bfloat16, device="cuda")
+        with pytest.raises(F.FavorError) as e:
+            F.favor_attention(q, q, q, om, feature_kind=kind)
+        assert e.value.code == -5
