@@ -31,6 +31,8 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD = dict(B=4, H=8, L=4096, d=64, M=256)
 VARIANTS = [("trig_bidir", 0, False), ("relu_bidir", 1, False), ("trig_causal", 0, True), ("relu_causal", 1, True)]
+# kernel launches per call of each variant: bidirectional = key states, merge, queries
+LAUNCHES = {"trig_bidir": 3, "relu_bidir": 3, "trig_causal": 1, "relu_causal": 1}
 N_SETS = 4
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "FAVOR fwd tokens/s (B·H·L/s) at L=4096,d=64,M=256; % of tensor/HBM roofline"
@@ -39,15 +41,11 @@ METRIC = "FAVOR fwd tokens/s (B·H·L/s) at L=4096,d=64,M=256; % of tensor/HBM r
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of each variant's kernel
 # at this workload, from one ncu capture (profiles/), with the SHA-1 of the kernel sources the
 # capture was taken with. A value whose sources have changed since is reported as null.
-TRAFFIC = {
-    "trig_bidir": (51392000, "f95d0ce2faf5715457f577f8bcf35140ab04a556"),
-    "relu_bidir": (51413248, "f95d0ce2faf5715457f577f8bcf35140ab04a556"),
-    "trig_causal": (51099392, "f95d0ce2faf5715457f577f8bcf35140ab04a556"),
-    "relu_causal": (51088640, "f95d0ce2faf5715457f577f8bcf35140ab04a556"),
-}
+TRAFFIC = {}
 KERNEL_SOURCES = ["linear_kernelized_attention_b200/csrc/ptx.cuh",
-                  "linear_kernelized_attention_b200/csrc/kernel_bidir.cuh",
-                  "linear_kernelized_attention_b200/csrc/kernel_causal.cuh"]
+                  "linear_kernelized_attention_b200/csrc/sincos_poly.cuh",
+                  "linear_kernelized_attention_b200/csrc/kernel_bidir_split.cuh",
+                  "linear_kernelized_attention_b200/csrc/kernel_causal_fs.cuh"]
 
 
 def kernel_sources_sha():
@@ -219,23 +217,21 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
-def run_lsweep(args):
+def lsweep_points(Ls, dev, stream, reps_budget=64):
     """Throughput against sequence length at B=1, H=16, d=64, M=256 (trig, bidirectional and
-    causal), L = 4096 .. 65536: one JSON line per (L, variant). Constant tokens/s across L is
-    linear scaling. Rotating input sets keep every point's reads above twice the L2 size."""
+    causal): one dict per (L, variant). Constant tokens/s across L is linear scaling. Rotating
+    input sets keep every point's reads above twice the L2 size; each point replays a CUDA graph
+    of one call per input set between CUDA events."""
     import numpy as np
     import torch
 
     import favor_inputs as fi
     import linear_kernelized_attention_b200 as F
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    stream = torch.cuda.Stream(device=dev)
-    torch.cuda.set_stream(stream)
     B, H, d, M = 1, 16, 64, 256
     G, R = fi.orf_gaussians(H, M, d, seed=0)
     omega = F.favor_orf_omega(torch.from_numpy(G).to(dev), torch.from_numpy(R).to(dev), M, dtype=torch.bfloat16)
-    for L in (4096, 8192, 16384, 32768, 65536):
+    points = []
+    for L in Ls:
         nbytes = 3 * B * H * L * d * 2
         nsets = max(1, int(np.ceil(2 * 126e6 / nbytes)))
         sets = []
@@ -255,7 +251,7 @@ def run_lsweep(args):
                     F.favor_attention(*sets[si], omega, out=out, feature_kind=0, causal=causal, stream=stream)
             g.replay()
             torch.cuda.synchronize()
-            reps = max(3, int(64 / nsets))
+            reps = max(3, int(reps_budget / nsets))
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             for _ in range(reps):
@@ -263,11 +259,23 @@ def run_lsweep(args):
             b.record(stream)
             torch.cuda.synchronize()
             us = 1e3 * a.elapsed_time(b) / (reps * nsets)
-            print(json.dumps({"lsweep": True, "L": L, "B": B, "H": H, "d": d, "M": M,
-                              "variant": "trig_causal" if causal else "trig_bidir", "us_per_launch": us,
-                              "tokens_per_s": B * H * L / (us * 1e-6), "input_sets": nsets}), flush=True)
+            points.append({"L": L, "B": B, "H": H, "d": d, "M": M,
+                           "variant": "trig_causal" if causal else "trig_bidir", "us_per_call": us,
+                           "tokens_per_s": B * H * L / (us * 1e-6), "input_sets": nsets})
             del g
         del sets
+    return points
+
+
+def run_lsweep(args):
+    """bench.py --lsweep: the L sweep 4096 .. 65536, one JSON line per (L, variant)."""
+    import torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    for pt in lsweep_points((4096, 8192, 16384, 32768, 65536), dev, stream):
+        print(json.dumps({"lsweep": True, **pt}), flush=True)
 
 
 def decode_bytes_per_call(B, H, d, M, kind):
@@ -459,6 +467,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-lsweep", action="store_true", help="leave the L = 4096 / 65536 points out of the bench line")
     ap.add_argument("--lsweep", action="store_true",
                     help="throughput against L (B=1, H=16, trig) instead of the bench line")
     ap.add_argument("--decode", action="store_true",
@@ -546,10 +555,20 @@ def main():
 
     clocks = ClockSampler(local)
     clocks.start()
+    # clock window: about a second of the same step replays, untimed, right before the timed
+    # region, so the clock record has samples under this load even when the timed region is
+    # shorter than the sampling interval; the timed region itself is sampled too
+    clocks.active.set()
+    t_win = time.perf_counter()
+    i = 0
+    while time.perf_counter() - t_win < 1.0:
+        for _ in range(50):
+            step_graphs[i % N_SETS].replay()
+            i += 1
+        torch.cuda.synchronize()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks.active.set()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(args.steps):
@@ -578,7 +597,14 @@ def main():
     tokens_step = len(variants) * B * H * L
     value = world * tokens_step / (ms * 1e-3)
 
-    # roofline of the dominant kernel (each variant is one kernel launch)
+    # linear scaling in L: B=1, H=16 trig at L = 4096 and 65536 (rank 0 only)
+    lsw = None
+    if rank == 0 and not args.no_lsweep:
+        lsw = lsweep_points((4096, 65536), dev, stream, reps_budget=16)
+        torch.cuda.set_stream(stream)
+
+    # roofline of the dominant variant (a causal call is one kernel launch; a bidirectional call
+    # is three: key states, merge, queries)
     peaks, peak_src = load_peaks()
     dom = max(per_variant, key=per_variant.get)
     kind = [vv[1] for vv in variants if vv[0] == dom][0]
@@ -625,9 +651,11 @@ def main():
             "config": {"workload": "favor_fwd_B4_H8_L4096_d64_M256", **W,
                        "variants": [vv[0] for vv in variants], "ms_per_launch": per_variant,
                        "l2": f"{N_SETS} rotating input sets ({N_SETS * 4 * B * H * L * d * 2 / 1e6:.0f} MB) > 2x L2",
-                       "parallelism": f"replica x{world} (independent heads per rank)"},
+                       "parallelism": f"replica x{world} (independent heads per rank)",
+                       "launches_per_call": LAUNCHES, "lsweep": lsw},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps * len(variants), "clocks": clocks.summary(),
+            "gpu_launches": args.steps * sum(LAUNCHES[vv[0]] for vv in variants),
+            "clocks": {**clocks.summary(), "window": "1 s of the same step replays right before the timed region, and the timed region"},
         }
         print(json.dumps(line), flush=True)
     del step_graphs, var_graphs

@@ -14,8 +14,6 @@
 #include "../../include/favor.h"
 #include "ptx.cuh"
 #include "kernels_f32.cuh"
-#include "kernel_bidir.cuh"
-#include "kernel_causal.cuh"
 #include "kernel_bidir_split.cuh"
 #include "kernel_causal_fs.cuh"
 #include "kernel_decode.cuh"
@@ -121,20 +119,6 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D bf16 tensor [n2][n1][64] with 128-byte rows, box {64, 128, 1}, 128-byte swizzle,
-// out-of-range rows read as zero and are not written.
-bool make_map_rows64(CUtensorMap* m, const void* ptr, uint64_t n1, uint64_t n2) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {64, n1, n2};
-  const cuuint64_t strides[2] = {128, 128 * n1};
-  const cuuint32_t box[3] = {64, 128, 1};
-  const cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // 3-D bf16 tensor [n2][n1][d] (d = 16, 32, 64 or 128 elements per row) read in boxes of
 // {64, 128, 1} with 128-byte swizzle. Columns past d and rows past n1 read as zero and are not
 // written; a row of d = 128 takes two boxes (columns 0 and 64).
@@ -180,24 +164,6 @@ int scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
   return cudaMallocFromPoolAsync(p, bytes, pool, st) == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
 
-// ------------------------------------------------------------------ bf16 bidirectional plan
-struct BidirPlan {
-  int P, Mpad, ntiles;
-};
-
-// One cluster of P CTAs per head, P a power of two (<= 8, <= tiles) chosen so that B*H*P fills
-// the SMs once. The key-phase state is reduced through distributed shared memory, so the
-// bidirectional path needs no global scratch.
-BidirPlan plan_bidir(int BH, int L, int M) {
-  BidirPlan pl{};
-  pl.Mpad = (M + 127) / 128 * 128;
-  pl.ntiles = (L + tc::kTile - 1) / tc::kTile;
-  int P = 1;
-  while (P < 8 && BH * P * 2 <= sm_count() && P * 2 <= pl.ntiles) P *= 2;
-  pl.P = P;
-  return pl;
-}
-
 int check_tc_shape(int d, int M, int kind, int causal) {
   if (d != 16 && d != 32 && d != 64 && d != 128) return FAVOR_ERR_UNSUPPORTED;
   if (kind == FAVOR_TRIG && M > 256) return FAVOR_ERR_UNSUPPORTED;
@@ -228,7 +194,9 @@ void plan_split_t(SplitPlan& pl, int BH, int L, int M) {
   pl.units_k = pl.npairs * pl.ntiles;
   pl.units_q = (long long)BH * pl.ntiles;
   const int sms = sm_count();
-  pl.Pk = (int)std::min<long long>(sms, pl.units_k);
+  // a pair's tiles spread over at most Pk / npairs + 2 runs; the merge weights at most
+  // bs::kMergeMaxSlots of them
+  pl.Pk = (int)std::min<long long>(std::min<long long>(sms, pl.units_k), (bs::kMergeMaxSlots - 2) * pl.npairs);
   pl.Pq = (int)std::min<long long>(sms, pl.units_q);
   const long long per = pl.units_k / pl.Pk;  // >= 1
   pl.smax = (int)std::min<long long>(pl.Pk, (pl.ntiles + per - 1) / per + 1);
@@ -252,7 +220,7 @@ bool plan_split(SplitPlan& pl, int BH, int L, int d, int M, int kind) {
   } else {
     if (dp == 64) plan_split_t<1, 64>(pl, BH, L, M); else plan_split_t<1, 128>(pl, BH, L, M);
   }
-  return pl.q_smem <= 232448;
+  return pl.q_smem <= 232448 && pl.smax <= bs::kMergeMaxSlots;
 }
 
 template <int KIND, int DP>
@@ -292,7 +260,21 @@ int launch_split_t(const SplitPlan& pl, const void* q, const void* k, const void
   mp.meta = meta;
   mp.img = img;
   mp.img_bytes = (long long)pl.img_bytes_head;
-  bs::k_bidir_merge<KIND, DP><<<dim3((unsigned)pl.npairs, bs::StateCfg<KIND, DP>::R / 32), 256, 0, st>>>(mp);
+  // the merge and the query kernel are launched with programmatic stream serialization: each may
+  // start while the kernel before it drains, and waits (griddepcontrol.wait) before reading its
+  // results
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)pl.npairs, bs::StateCfg<KIND, DP>::R / 32, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = st;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, bs::k_bidir_merge<KIND, DP>, mp) != cudaSuccess) return FAVOR_ERR_CUDA;
+  }
 
   bs::QueryParams qp{};
   qp.H = H;
@@ -310,7 +292,16 @@ int launch_split_t(const SplitPlan& pl, const void* q, const void* k, const void
   qp.off_misc = pl.q_off_misc;
   auto kq = bs::k_bidir_query<KIND, DP>;
   if (ensure_smem_attr(reinterpret_cast<const void*>(kq), pl.q_smem) != FAVOR_OK) return FAVOR_ERR_CUDA;
-  kq<<<pl.Pq, bs::kThreads, pl.q_smem, st>>>(mq, mom, mo, qp);
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.Pq, 1, 1);
+    cfg.blockDim = dim3(bs::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = pl.q_smem;
+    cfg.stream = st;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kq, mq, mom, mo, qp) != cudaSuccess) return FAVOR_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
 
@@ -331,95 +322,6 @@ int launch_bidir_split(const void* q, const void* k, const void* v, const void* 
                      : launch_split_t<1, 128>(pl, q, k, v, omega, out, BH, H, L, d, M, ws, st);
   cudaFreeAsync(ws, st);
   return rc;
-}
-
-int launch_bidir_bf16(const void* q, const void* k, const void* v, const void* omega, void* out,
-                      int B, int H, int L, int M, int kind, cudaStream_t st) {
-  const int BH = B * H;
-  if (BH > 65535 * 8) return FAVOR_ERR_UNSUPPORTED;
-  const BidirPlan pl = plan_bidir(BH, L, M);
-  CUtensorMap mq, mk, mv, mo, mom;
-  if (!make_map_rows64(&mq, q, L, BH) || !make_map_rows64(&mk, k, L, BH) ||
-      !make_map_rows64(&mv, v, L, BH) || !make_map_rows64(&mo, out, L, BH) ||
-      !make_map_rows64(&mom, omega, M, H))
-    return FAVOR_ERR_CUDA;
-  tc::BidirParams prm{};
-  prm.BH = BH;
-  prm.H = H;
-  prm.L = L;
-  prm.M = M;
-  prm.Mpad = pl.Mpad;
-  prm.P = pl.P;
-  prm.ntiles = pl.ntiles;
-  const uint32_t smem = tc::bidir_smem_bytes(pl.Mpad);
-  // Trig keys use 32-token slices; ReLU uses 64-token slices when its state (<= 2 blocks of
-  // 128 features) leaves TMEM room for them.
-  auto kern = kind == FAVOR_TRIG ? tc::favor_bidir_tc<0, 32>
-              : (pl.Mpad <= 256 ? tc::favor_bidir_tc<1, 64> : tc::favor_bidir_tc<1, 32>);
-  if (ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)smem) != FAVOR_OK) return FAVOR_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(BH * pl.P, 1, 1);
-  cfg.blockDim = dim3(tc::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = pl.P;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mom, mo, prm) == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
-}
-
-// ------------------------------------------------------------------ bf16 causal
-// Angles per CTA: 64 (trig; ReLU with M <= 256) or 128 (ReLU with M > 256).
-int causal_angles(int M, int kind) { return kind == FAVOR_RELU && M > 256 ? 128 : 64; }
-
-// CTAs per head; 3 rounds up to 4 so that the cluster's row ownership (rows of warp quarter q go
-// to CTA q % G) is balanced.
-int causal_blocks(int M, int kind) {
-  const int na = causal_angles(M, kind);
-  const int G = (M + na - 1) / na;
-  return G == 3 ? 4 : G;
-}
-
-int launch_causal_bf16(const void* q, const void* k, const void* v, const void* omega, void* out,
-                       int B, int H, int L, int M, int kind, cudaStream_t st) {
-  const int BH = B * H;
-  const int G = causal_blocks(M, kind);
-  if (G < 1 || G > 4) return FAVOR_ERR_UNSUPPORTED;
-  if ((long long)BH * G > INT_MAX) return FAVOR_ERR_UNSUPPORTED;
-  CUtensorMap mq, mk, mv, mom;
-  if (!make_map_rows64(&mq, q, L, BH) || !make_map_rows64(&mk, k, L, BH) ||
-      !make_map_rows64(&mv, v, L, BH) || !make_map_rows64(&mom, omega, M, H))
-    return FAVOR_ERR_CUDA;
-  tc::CausalParams prm{};
-  prm.BH = BH;
-  prm.H = H;
-  prm.L = L;
-  prm.M = M;
-  prm.G = G;
-  prm.nch = (L + tc::kTile - 1) / tc::kTile;
-  const uint32_t smem = tc::causal_smem_bytes();
-  auto kern = kind == FAVOR_TRIG ? tc::favor_causal_tc<0, 64>
-              : (causal_angles(M, kind) == 64 ? tc::favor_causal_tc<1, 64> : tc::favor_causal_tc<1, 128>);
-  if (ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)smem) != FAVOR_OK) return FAVOR_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(BH * G, 1, 1);
-  cfg.blockDim = dim3(tc::kThreadsC, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = G;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mom, prm, static_cast<__nv_bfloat16*>(out)) == cudaSuccess
-             ? FAVOR_OK
-             : FAVOR_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ bf16 causal, feature split
@@ -706,7 +608,7 @@ int favor_attention_chunked(const void* q, const void* k, const void* v, const v
   if ((rc = check_tc_shape(d, M, feature_kind, causal)) != FAVOR_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (causal) {
-    if (chunk != 0 && chunk != tc::kTile) return FAVOR_ERR_UNSUPPORTED;
+    if (chunk != 0 && chunk != cf::kTile) return FAVOR_ERR_UNSUPPORTED;
     return launch_causal_fs(q, k, v, omega, out, B, H, L, d, M, feature_kind, st);
   }
   return launch_bidir_split(q, k, v, omega, out, B, H, L, d, M, feature_kind, st);

@@ -174,13 +174,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
+  pdl_launch_dependents();  // the merge may be scheduled; it waits for this grid's results
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && n > 0) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_om);
+    // ------------------------------------------------------------ TMA producer (whole warp; the
+    // elected lane issues the copies)
+    if (n > 0) {
+      const bool leader = elect_one();
+      if (leader) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_om);
+      }
       int issued = 0, pk_issued = 0;
       for (int t = 0; t < n; ++t) {
         const long long x = u0 + t, pr = x / nt;
@@ -188,19 +193,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bh = (int)(pr / p.nab), ab = (int)(pr % p.nab), h = bh % p.H;
         if (first_of_pair(t)) {
           if (pk >= 2 && !mbar_wait(bar(ms->om_free[pk & 1]), ((pk >> 1) - 1) & 1, abort_flag)) break;
-          mbar_arrive_expect_tx(bar(ms->om_full[pk & 1]), C::kOmB);
-          for (int kb = 0; kb < NCB; ++kb)
-            tma_load_3d(s_om + (pk & 1) * C::kOmB + kb * kBoxB, &tm_om, bar(ms->om_full[pk & 1]), kb * 64, ab * 128, h);
+          if (leader) {
+            mbar_arrive_expect_tx(bar(ms->om_full[pk & 1]), C::kOmB);
+            for (int kb = 0; kb < NCB; ++kb)
+              tma_load_3d(s_om + (pk & 1) * C::kOmB + kb * kBoxB, &tm_om, bar(ms->om_full[pk & 1]), kb * 64, ab * 128,
+                          h);
+          }
           pk_issued = pk + 1;
         }
         const int s = t % NS;
         if (t >= NS && !mbar_wait(bar(ms->kv_empty[s]), ((t / NS) - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(ms->kv_full[s]), 2 * NCB * kBoxB);
         const uint32_t st = s_stage + s * C::kStageB;
         const int row = (int)(x % nt) * kTile;
-        for (int kb = 0; kb < NCB; ++kb) {
-          tma_load_3d(st + kb * kBoxB, &tm_v, bar(ms->kv_full[s]), kb * 64, row, bh);
-          tma_load_3d(st + (NCB + 1 + kb) * kBoxB, &tm_k, bar(ms->kv_full[s]), kb * 64, row, bh);
+        if (leader) {
+          mbar_arrive_expect_tx(bar(ms->kv_full[s]), 2 * NCB * kBoxB);
+          for (int kb = 0; kb < NCB; ++kb) {
+            tma_load_3d(st + kb * kBoxB, &tm_v, bar(ms->kv_full[s]), kb * 64, row, bh);
+            tma_load_3d(st + (NCB + 1 + kb) * kBoxB, &tm_k, bar(ms->kv_full[s]), kb * 64, row, bh);
+          }
         }
         issued = t + 1;
       }
@@ -214,8 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n > 0) {
+    // ------------------------------------------------------------ MMA issuer (whole warp; the
+    // elected lane issues the MMAs and commits)
+    if (n > 0) {
+      const bool leader = elect_one();
       const uint32_t id1 = idesc_f16(128, 64, 1, 1, 0, 0);
       const uint32_t id2 = idesc_f16(128, NV, 1, 1, 0, 1);
       const int nitems = 2 * n;
@@ -231,23 +243,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t a0 = sdesc_sw128(s_om + (pk & 1) * C::kOmB, 16, 1024);
         const uint64_t b0 = sdesc_sw128(s_stage + s * C::kStageB + (NCB + 1) * kBoxB + hf * 64 * kRowB, 16, 1024);
         const uint32_t d = tmem + C::kUcol + b * 64;
+        if (leader) {
 #pragma unroll
-        for (int kb = 0; kb < NCB; ++kb)
+          for (int kb = 0; kb < NCB; ++kb)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t off = uint64_t((kb * kBoxB + kk * 32) >> 4);
-            mma_ss(d, a0 + off, b0 + off, id1, (kb | kk) ? 1u : 0u);
-          }
-        mma_commit(bar(ms->u_full[b]));
-        if (hf == 1 && last_of_pair(t)) mma_commit(bar(ms->om_free[pk & 1]));
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t off = uint64_t((kb * kBoxB + kk * 32) >> 4);
+              mma_ss(d, a0 + off, b0 + off, id1, (kb | kk) ? 1u : 0u);
+            }
+          mma_commit(bar(ms->u_full[b]));
+          if (hf == 1 && last_of_pair(t)) mma_commit(bar(ms->om_free[pk & 1]));
+        }
+        __syncwarp();
         return true;
       };
       auto write_meta_max = [&](int pk) {
         float mx = 0.f;
         for (int w = 0; w < 8; ++w) mx = fmaxf(mx, ms->redmax[pk & 1][w]);
         const long long sl = slot_of(p0 + pk);
-        p.meta[sl * 2 + 1] = mx;
-        if (KIND == 1) p.meta[sl * 2] = 0.f;
+        if (leader) {
+          p.meta[sl * 2 + 1] = mx;
+          if (KIND == 1) p.meta[sl * 2] = 0.f;
+        }
       };
       for (int it = 0; ok && it < NBUF && it < nitems; ++it) ok = mma1(it);
       for (int it = 0; ok && it < nitems; ++it) {
@@ -264,19 +281,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t vd =
             sdesc_sw128(s_stage + s * C::kStageB, kBoxB, 1024) + uint64_t((hf * 64 * kRowB) >> 4);
         const uint32_t ub = tmem + C::kUcol + b * 64;
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = vd + uint64_t((kk * 16 * kRowB) >> 4);
-          const uint32_t acc = (fresh && kk == 0) ? 0u : 1u;
-          const uint32_t col = 32 * (kk >> 1) + 8 * (kk & 1);
-          mma_ts(tmem, ub + col, bd, id2, acc);
-          if (KIND == 0) mma_ts(tmem + NV, ub + 16 + col, bd, id2, acc);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = vd + uint64_t((kk * 16 * kRowB) >> 4);
+            const uint32_t acc = (fresh && kk == 0) ? 0u : 1u;
+            const uint32_t col = 32 * (kk >> 1) + 8 * (kk & 1);
+            mma_ts(tmem, ub + col, bd, id2, acc);
+            if (KIND == 0) mma_ts(tmem + NV, ub + 16 + col, bd, id2, acc);
+          }
+          mma_commit(bar(ms->buf_free[b]));
+          if (hf == 1) {
+            mma_commit(bar(ms->kv_empty[s]));
+            if (last_of_pair(t)) mma_commit(bar(ms->s_done));
+          }
         }
-        mma_commit(bar(ms->buf_free[b]));
-        if (hf == 1) {
-          mma_commit(bar(ms->kv_empty[s]));
-          if (last_of_pair(t)) mma_commit(bar(ms->s_done));
-        }
+        __syncwarp();
         const int nx = it + NBUF;
         if (nx < nitems) {
           if (!(ok = mbar_wait(bar(ms->buf_free[b]), (it / NBUF) & 1, abort_flag))) break;
@@ -287,7 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int pk_last = (int)(pair_of(n - 1) - p0);
         if (mbar_wait(bar(ms->s_free), pk_last & 1, abort_flag)) write_meta_max(pk_last);
       }
-      mma_commit(bar(ms->drain));
+      if (leader) mma_commit(bar(ms->drain));
+      __syncwarp();
       mbar_wait(bar(ms->drain), 0, nullptr, kWaitLimitCycles / 8);
     }
     __syncwarp();
@@ -398,8 +419,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             float s0, c0, s1, c1;
             sincos_mixed<kPolyMask>(2 * e, __uint_as_float(u[2 * e]), s0, c0);
             sincos_mixed<kPolyMask>(2 * e + 1, __uint_as_float(u[2 * e + 1]), s1, c1);
+#ifdef FAVOR_PACK_TRUNC
+            cp[e] = pack_hi16(c0, c1);
+            sp[e] = pack_hi16(s0, s1);
+#else
             cp[e] = pack_bf16x2(c0, c1);
             sp[e] = pack_bf16x2(s0, s1);
+#endif
           }
           tmem_st16(ub + 32 * c, cp);
           tmem_st16(ub + 32 * c + 16, sp);
@@ -490,43 +516,67 @@ __device__ __forceinline__ uint32_t img_byte(int f, int n) {
 }
 
 // One block per (pair, 32 state rows). Trig feature order within a 128-angle block: 32-angle
-// groups of [cos 32 | sin 32], matching the query kernel's packing.
+// groups of [cos 32 | sin 32], matching the query kernel's packing. The first warp turns the
+// head's slot metadata into per-slot weights in shared memory; then every thread sums its
+// elements over the pair's slots with all loads of an element in flight together.
+constexpr int kMergeMaxSlots = 64;  // slots of one head (nab * smax) the merge can weight
+
 template <int KIND, int DP>
 __global__ void __launch_bounds__(256) k_bidir_merge(const MergeParams p) {
   constexpr int NV = DP + 16, R = KIND == 0 ? 256 : 128, FB = R;
+  __shared__ float wts[kMergeMaxSlots];
+  __shared__ float scale_s;
+  pdl_launch_dependents();  // the query kernel may start its projections
+  pdl_wait();               // the key-state partials are complete
   const long long pr = blockIdx.x;
   const int rb = blockIdx.y;
   const long long bh = pr / p.nab;
   const int ab = (int)(pr % p.nab);
-  // the head's reference and the bound of its merged state
-  float cmax = -INFINITY;
-  for (int a2 = 0; a2 < p.nab; ++a2) {
-    const long long q2 = bh * p.nab + a2;
-    const int ns = nslots(q2, p);
-    for (int s = 0; s < ns; ++s) cmax = fmaxf(cmax, p.meta[(q2 * p.smax + s) * 2]);
-  }
-  float bound = 0.f;
-  for (int a2 = 0; a2 < p.nab; ++a2) {
-    const long long q2 = bh * p.nab + a2;
-    const int ns = nslots(q2, p);
-    for (int s = 0; s < ns; ++s) {
-      const float* m = p.meta + (q2 * p.smax + s) * 2;
-      bound += (KIND == 0 ? __expf(m[0] - cmax) : 1.f) * m[1];
+  if (threadIdx.x < 32) {
+    // the head's reference (max over its slots) and the bound of its merged state
+    const int lane = threadIdx.x;
+    float cmax = -INFINITY;
+    for (int a2 = 0; a2 < p.nab; ++a2) {
+      const long long q2 = bh * p.nab + a2;
+      const int ns = nslots(q2, p);
+      for (int s = lane; s < ns; s += 32) cmax = fmaxf(cmax, KIND == 0 ? p.meta[(q2 * p.smax + s) * 2] : 0.f);
     }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+    float bound = 0.f;
+    for (int a2 = 0; a2 < p.nab; ++a2) {
+      const long long q2 = bh * p.nab + a2;
+      const int ns = nslots(q2, p);
+      for (int s = lane; s < ns; s += 32) {
+        const float* m = p.meta + (q2 * p.smax + s) * 2;
+        const float w = KIND == 0 ? __expf(m[0] - cmax) : 1.f;
+        bound += w * m[1];
+        if (a2 == ab && s < kMergeMaxSlots) wts[s] = w;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) bound += __shfl_xor_sync(0xffffffffu, bound, o);
+    if (lane == 0) scale_s = (KIND == 0 && bound > 0.f) ? exp2f(14.f - ceilf(log2f(bound))) : 1.f;
   }
-  const float scale = (KIND == 0 && bound > 0.f) ? exp2f(14.f - ceilf(log2f(bound))) : 1.f;
-  const int ns = nslots(pr, p);
+  __syncthreads();
+  const float scale = scale_s;
+  const int ns = min(nslots(pr, p), kMergeMaxSlots);
   uint8_t* img = p.img + bh * p.img_bytes;
+  const float* part = p.part + pr * p.smax * (long long)(DP + 1) * R;
   for (int e = threadIdx.x; e < 32 * NV; e += blockDim.x) {
     const int rl = e & 31, nn = e >> 5;
     const int r = rb * 32 + rl;
     float v = 0.f;
     if (nn <= DP) {
-      for (int s = 0; s < ns; ++s) {
-        const long long sl = pr * p.smax + s;
-        const float w = KIND == 0 ? __expf(p.meta[sl * 2] - cmax) : 1.f;
-        v = fmaf(w, p.part[(sl * (DP + 1) + nn) * R + r], v);
+      const float* src = part + (long long)nn * R + r;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      int s = 0;
+      for (; s + 4 <= ns; s += 4) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) acc[t] = fmaf(wts[s + t], src[(long long)(s + t) * (DP + 1) * R], acc[t]);
       }
+      for (; s < ns; ++s) acc[0] = fmaf(wts[s], src[(long long)s * (DP + 1) * R], acc[0]);
+      v = (acc[0] + acc[1]) + (acc[2] + acc[3]);
     }
     const int a = KIND == 0 ? (r & 127) : r;
     if (ab * 128 + a >= p.M) v = 0.f;  // padded angle
@@ -621,32 +671,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = ms->tmem_base;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && n > 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_om);
-      tma_prefetch_desc(&tm_out);
+    // ------------------------------------------------------------ TMA producer (whole warp; the
+    // elected lane issues the copies)
+    if (n > 0) {
+      const bool leader = elect_one();
+      if (leader) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_om);
+        tma_prefetch_desc(&tm_out);
+      }
       int issued = 0, heads = 0;
       for (int t = 0; t < n; ++t) {
         const long long x = u0 + t, bh = x / nt;
         const int s = t & 1;
         if (t >= 2 && !mbar_wait(bar(ms->q_empty[s]), ((t >> 1) - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(ms->q_full[s]), NCB * kBoxB);
-        for (int kb = 0; kb < NCB; ++kb)
-          tma_load_3d(s_q + (s * NCB + kb) * kBoxB, &tm_q, bar(ms->q_full[s]), kb * 64, (int)(x % nt) * kTile, (int)bh);
+        if (leader) {
+          mbar_arrive_expect_tx(bar(ms->q_full[s]), NCB * kBoxB);
+          for (int kb = 0; kb < NCB; ++kb)
+            tma_load_3d(s_q + (s * NCB + kb) * kBoxB, &tm_q, bar(ms->q_full[s]), kb * 64, (int)(x % nt) * kTile,
+                        (int)bh);
+        }
         issued = t + 1;
         if (first_of_head(t)) {
           const int hk = (int)(bh - h0);
+          if (hk == 0) pdl_wait();  // the merge has written the state images
           if (hk >= 1 && !mbar_wait(bar(ms->head_free), (hk - 1) & 1, abort_flag)) break;
-          mbar_arrive_expect_tx(bar(ms->head_full), p.om_bytes + p.img_bytes);
           const int h = (int)(bh % p.H);
-          for (int ab = 0; ab < nab; ++ab)
-            for (int kb = 0; kb < NCB; ++kb)
-              tma_load_3d(s_om + (ab * NCB + kb) * kBoxB, &tm_om, bar(ms->head_full), kb * 64, ab * 128, h);
           const uint8_t* src = p.img + bh * p.img_bytes;
-          for (int off = 0; off < p.img_bytes; off += 32768) {
-            const int sz = min(32768, p.img_bytes - off);
-            bulk_load(s_img + off, src + off, sz, bar(ms->head_full));
+          if (leader) {
+            mbar_arrive_expect_tx(bar(ms->head_full), p.om_bytes + p.img_bytes);
+            for (int ab = 0; ab < nab; ++ab)
+              for (int kb = 0; kb < NCB; ++kb)
+                tma_load_3d(s_om + (ab * NCB + kb) * kBoxB, &tm_om, bar(ms->head_full), kb * 64, ab * 128, h);
+            for (int off = 0; off < p.img_bytes; off += 32768) {
+              const int sz = min(32768, p.img_bytes - off);
+              bulk_load(s_img + off, src + off, sz, bar(ms->head_full));
+            }
           }
           heads = hk + 1;
         }
@@ -660,8 +720,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n > 0) {
+    // ------------------------------------------------------------ MMA issuer (whole warp; the
+    // elected lane issues the MMAs and commits)
+    if (n > 0) {
+      const bool leader = elect_one();
       const uint32_t id1 = idesc_f16(128, 128, 1, 1, 0, 0);
       const uint32_t fmt = KIND == 0 ? 0u : 1u;  // fp16 (trig) or bf16 (ReLU) state operands
       const uint32_t id2 = idesc_f16(128, NV, fmt, fmt, 0, 0);
@@ -679,14 +741,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= 2 && !mbar_wait(bar(ms->buf_free[b]), ((j - 2) >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint64_t q0 = sdesc_sw128(s_q + s * NCB * kBoxB, 16, 1024);
+        if (leader) {
 #pragma unroll
-        for (int kb = 0; kb < NCB; ++kb)
+          for (int kb = 0; kb < NCB; ++kb)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + b * 128, q0 + uint64_t((kb * kBoxB + kk * 32) >> 4),
-                   om0 + uint64_t(((ab * NCB + kb) * kBoxB + kk * 32) >> 4), id1, (kb | kk) ? 1u : 0u);
-        mma_commit(bar(ms->u_full[b]));
-        if (ab == nab - 1) mma_commit(bar(ms->q_empty[s]));
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tmem + b * 128, q0 + uint64_t((kb * kBoxB + kk * 32) >> 4),
+                     om0 + uint64_t(((ab * NCB + kb) * kBoxB + kk * 32) >> 4), id1, (kb | kk) ? 1u : 0u);
+          mma_commit(bar(ms->u_full[b]));
+          if (ab == nab - 1) mma_commit(bar(ms->q_empty[s]));
+        }
+        __syncwarp();
         return true;
       };
       int nx = 0;  // next item whose projection is to be issued
@@ -697,17 +762,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ab == 0 && t >= NBN && !(ok = mbar_wait(bar(ms->num_empty[nb]), ((t / NBN) - 1) & 1, abort_flag))) break;
         tc_fence_after();
         const uint32_t dn = tmem + C::kNumCol + nb * NV;
-#pragma unroll
-        for (int kk = 0; kk < FB / 16; ++kk) {
-          const int f = ab * FB + 16 * kk;
-          const uint64_t bd = img0 + uint64_t(((f >> 6) * (NV * kRowB) + ((f & 63) >> 4) * 32) >> 4);
-          const uint32_t acol = KIND == 0 ? 8 * kk : 64 * (kk >> 2) + 8 * (kk & 3);
-          mma_ts(dn, tmem + b * 128 + acol, bd, id2, (ab | kk) ? 1u : 0u);
-        }
-        mma_commit(bar(ms->buf_free[b]));
         const bool head_end = ab == nab - 1 && last_of_head(t);
-        if (ab == nab - 1) mma_commit(bar(ms->num_full[nb]));
-        if (head_end) mma_commit(bar(ms->head_free));
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < FB / 16; ++kk) {
+            const int f = ab * FB + 16 * kk;
+            const uint64_t bd = img0 + uint64_t(((f >> 6) * (NV * kRowB) + ((f & 63) >> 4) * 32) >> 4);
+            const uint32_t acol = KIND == 0 ? 8 * kk : 64 * (kk >> 2) + 8 * (kk & 3);
+            mma_ts(dn, tmem + b * 128 + acol, bd, id2, (ab | kk) ? 1u : 0u);
+          }
+          mma_commit(bar(ms->buf_free[b]));
+          if (ab == nab - 1) mma_commit(bar(ms->num_full[nb]));
+          if (head_end) mma_commit(bar(ms->head_free));
+        }
+        __syncwarp();
         // projections ahead: two items in flight, and none past a head change until the head's
         // last state product has been issued (the next head's Omega and image replace these)
         while (ok && nx < nit && nx <= j + 2) {
@@ -716,7 +784,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mma1(nx++);
         }
       }
-      mma_commit(bar(ms->drain));
+      if (leader) mma_commit(bar(ms->drain));
+      __syncwarp();
       mbar_wait(bar(ms->drain), 0, nullptr, kWaitLimitCycles / 8);
     }
     __syncwarp();

@@ -227,27 +227,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint64_t kKStep = (16 * kRowB) >> 4;  // 16 rows of an MN-major operand
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_q);
-      mbar_arrive_expect_tx(bar(ms->om_full), kTileB);
-      tma_load_3d(base + kC_OM, &tm_om, bar(ms->om_full), 0, g * NA, h);
+    // ------------------------------------------------------------ TMA producer (whole warp; the
+    // elected lane issues the copies)
+    {
+      const bool leader = elect_one();
+      if (leader) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_q);
+        mbar_arrive_expect_tx(bar(ms->om_full), kTileB);
+        tma_load_3d(base + kC_OM, &tm_om, bar(ms->om_full), 0, g * NA, h);
+      }
       int k_issued = 0, v_issued = 0, q_issued = 0;
       for (int c = 0; c < nch; ++c) {
         const int s = c & 1;
         if (c >= 1 && !mbar_wait(bar(ms->k_empty), (c - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(ms->k_full), kTileB);
-        tma_load_3d(base + kC_K, &tm_k, bar(ms->k_full), 0, c * kTile, bh);
+        if (leader) {
+          mbar_arrive_expect_tx(bar(ms->k_full), kTileB);
+          tma_load_3d(base + kC_K, &tm_k, bar(ms->k_full), 0, c * kTile, bh);
+        }
         k_issued = c + 1;
         if (c >= 2 && !mbar_wait(bar(ms->v_empty[s]), ((c >> 1) - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(ms->v_full[s]), kTileB);
-        tma_load_3d(base + kC_V + s * kTileB, &tm_v, bar(ms->v_full[s]), 0, c * kTile, bh);
+        if (leader) {
+          mbar_arrive_expect_tx(bar(ms->v_full[s]), kTileB);
+          tma_load_3d(base + kC_V + s * kTileB, &tm_v, bar(ms->v_full[s]), 0, c * kTile, bh);
+        }
         v_issued = c + 1;
         if (c >= 1 && !mbar_wait(bar(ms->q_empty), (c - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(ms->q_full), kTileB);
-        tma_load_3d(base + kC_Q, &tm_q, bar(ms->q_full), 0, c * kTile, bh);
+        if (leader) {
+          mbar_arrive_expect_tx(bar(ms->q_full), kTileB);
+          tma_load_3d(base + kC_Q, &tm_q, bar(ms->q_full), 0, c * kTile, bh);
+        }
         q_issued = c + 1;
       }
       // On an abort, let the copies already issued land before the CTA can exit.
@@ -262,8 +272,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ issuer A: U_K, S and z
-    if (lane == 0) {
+    // ------------------------------------------------------------ issuer A: U_K, S and z (whole
+    // warp; the elected lane issues)
+    {
+      const bool leader = elect_one();
       const uint64_t d_om = sdesc_sw128(base + kC_OM, 16, 1024);
       const uint64_t d_k = sdesc_sw128(base + kC_K, 16, 1024);
       const uint64_t d_phk_a = sdesc_sw128(base + kC_PHK, kTileB, 1024);  // MN-major A of S, z
@@ -274,10 +286,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(bar(ms->k_full), c & 1, abort_flag)) return false;
         if (c > 0 && !mbar_wait(bar(ms->uk_free), (c - 1) & 1, abort_flag)) return false;
         tc_fence_after();
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + kT_B, d_k + 2 * kk, d_om + 2 * kk, id_uk, kk > 0 ? 1u : 0u);
-        mma_commit(bar(ms->uk_full));
-        mma_commit(bar(ms->k_empty));  // the K tile has been read
+          for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + kT_B, d_k + 2 * kk, d_om + 2 * kk, id_uk, kk > 0 ? 1u : 0u);
+          mma_commit(bar(ms->uk_full));
+          mma_commit(bar(ms->k_empty));  // the K tile has been read
+        }
+        __syncwarp();
         return true;
       };
       bool ok = mbar_wait(bar(ms->om_full), 0, abort_flag) && (nch == 0 || uk(0));
@@ -290,24 +305,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t a = d_phk_a + uint64_t(((c & 1) * kPhkB) >> 4);
         const bool use_vw = KIND == 0 && sm->fb[c & (kMeta - 1)];
         const uint64_t bvw = use_vw ? d_vw : d_v0 + uint64_t(((c & 1) * kTileB) >> 4);
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
-          mma_ss(tmem + kT_S, a + kk * kKStep, bvw + kk * kKStep, id_s, acc);
-          mma_ss(tmem + kT_S + 64, a + kk * kKStep, d_wr + uint64_t(((kk >> 2) * 2048 + (kk & 3) * 32) >> 4), id_z,
-                 acc);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
+            mma_ss(tmem + kT_S, a + kk * kKStep, bvw + kk * kKStep, id_s, acc);
+            mma_ss(tmem + kT_S + 64, a + kk * kKStep, d_wr + uint64_t(((kk >> 2) * 2048 + (kk & 3) * 32) >> 4),
+                   id_z, acc);
+          }
+          mma_commit(bar(ms->s_done));
+          mma_commit(bar(ms->v_empty[c & 1]));  // the V tile has been read
         }
-        mma_commit(bar(ms->s_done));
-        mma_commit(bar(ms->v_empty[c & 1]));  // the V tile has been read
+        __syncwarp();
         if (c + 1 < nch && !(ok = uk(c + 1))) break;
       }
-      mma_commit(bar(ms->drain_a));
+      if (leader) mma_commit(bar(ms->drain_a));
+      __syncwarp();
       mbar_wait(bar(ms->drain_a), 0, nullptr, kWaitLimitCycles / 8);
     }
     __syncwarp();
   } else if (warp == 2) {
     // ------------------------------------------------------------ issuer B: U_Q, P, inter, intra
-    if (lane == 0) {
+    // (whole warp; the elected lane issues)
+    {
+      const bool leader = elect_one();
       const uint64_t d_om = sdesc_sw128(base + kC_OM, 16, 1024);
       const uint64_t d_q = sdesc_sw128(base + kC_Q, 16, 1024);
       const uint64_t d_v0 = sdesc_sw128(base + kC_V, kTileB, 1024);
@@ -319,11 +340,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(bar(ms->q_full), c & 1, abort_flag)) return false;
         if (c >= 2 && !mbar_wait(bar(ms->slot_free[c & 1]), ((c >> 1) - 1) & 1, abort_flag)) return false;
         tc_fence_after();
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + kT_A + (c & 1) * 64, d_q + 2 * kk, d_om + 2 * kk, id_uk, kk > 0 ? 1u : 0u);
-        mma_commit(bar(ms->uq_full[c & 1]));
-        mma_commit(bar(ms->q_empty));
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + kT_A + (c & 1) * 64, d_q + 2 * kk, d_om + 2 * kk, id_uk, kk > 0 ? 1u : 0u);
+          mma_commit(bar(ms->uq_full[c & 1]));
+          mma_commit(bar(ms->q_empty));
+        }
+        __syncwarp();
         return true;
       };
       bool ok = mbar_wait(bar(ms->om_full), 0, abort_flag) && (nch == 0 || uq(0)) && (nch < 2 || uq(1));
@@ -335,36 +359,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c >= 1 && !(ok = mbar_wait(bar(ms->pr_free), (c - 1) & 1, abort_flag))) break;
         tc_fence_after();
         const uint64_t bk = d_phk_b + uint64_t(((c & 1) * kPhkB) >> 4);
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < NKS; ++kk)
-          mma_ts(tmem + kT_PR, slot + 8 * kk, bk + uint64_t(((kk >> 2) * kTileB + (kk & 3) * 32) >> 4), id_p,
-                 kk > 0 ? 1u : 0u);
-        mma_commit(bar(ms->p_full));
-        mma_commit(bar(ms->phik_free[c & 1]));
+          for (int kk = 0; kk < NKS; ++kk)
+            mma_ts(tmem + kT_PR, slot + 8 * kk, bk + uint64_t(((kk >> 2) * kTileB + (kk & 3) * 32) >> 4), id_p,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(bar(ms->p_full));
+          mma_commit(bar(ms->phik_free[c & 1]));
+        }
+        __syncwarp();
         // inter(c) = phi(Q) S_img and phi(Q).z
         if (!(ok = mbar_wait(bar(ms->img_full), c & 1, abort_flag))) break;
         tc_fence_after();
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < NKS; ++kk) {
-          mma_ts(tmem + kT_IN, slot + 8 * kk, d_img + kk * kKStep, id_in, kk > 0 ? 1u : 0u);
-          mma_ts(tmem + kT_IN + 64, slot + 8 * kk, d_zr + uint64_t(((kk >> 2) * 2048 + (kk & 3) * 32) >> 4),
-                 id_qz, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < NKS; ++kk) {
+            mma_ts(tmem + kT_IN, slot + 8 * kk, d_img + kk * kKStep, id_in, kk > 0 ? 1u : 0u);
+            mma_ts(tmem + kT_IN + 64, slot + 8 * kk, d_zr + uint64_t(((kk >> 2) * 2048 + (kk & 3) * 32) >> 4),
+                   id_qz, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(ms->img_free));
+          mma_commit(bar(ms->slot_free[c & 1]));
         }
-        mma_commit(bar(ms->img_free));
-        mma_commit(bar(ms->slot_free[c & 1]));
+        __syncwarp();
         // intra(c) = P16 V_c
         if (!(ok = mbar_wait(bar(ms->p16_full), c & 1, abort_flag))) break;
         tc_fence_after();
         const uint64_t bv = d_v0 + uint64_t(((c & 1) * kTileB) >> 4);
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + kT_PR + 64, tmem + kT_PR + 8 * kk, bv + kk * kKStep, id_it, kk > 0 ? 1u : 0u);
-        mma_commit(bar(ms->o_full));
-        mma_commit(bar(ms->v_empty[c & 1]));  // the V tile has been read
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + kT_PR + 64, tmem + kT_PR + 8 * kk, bv + kk * kKStep, id_it, kk > 0 ? 1u : 0u);
+          mma_commit(bar(ms->o_full));
+          mma_commit(bar(ms->v_empty[c & 1]));  // the V tile has been read
+        }
+        __syncwarp();
         // U_Q(c + 2) into this chunk's slot
         if (c + 2 < nch && !(ok = uq(c + 2))) break;
       }
-      mma_commit(bar(ms->drain_b));
+      if (leader) mma_commit(bar(ms->drain_b));
+      __syncwarp();
       mbar_wait(bar(ms->drain_b), 0, nullptr, kWaitLimitCycles / 8);
     }
     __syncwarp();

@@ -1,7 +1,7 @@
 """bf16 tensor-core path, causal: CUDA output vs the fp64 oracle on the same inputs.
 
-The causal kernel splits the features of a head over a cluster of G CTAs (G = 1, 2, 4) and
-scans 128-token chunks. Sizes cover one and many chunks, ragged tails, each cluster size, both
+The causal kernel splits the features of a head over a cluster of G CTAs of 64 angles each
+(G = 1, 2, 4, 8) and scans 128-token chunks. Sizes cover one and many chunks, ragged tails, each cluster size, both
 feature maps, padded feature counts, heavy-norm keys (the stabiliser's per-row references),
 the bench workload and a 65536-token sequence.
 """
@@ -28,9 +28,9 @@ def _run(case, kind, chunk=0):
     (1, 1, 1, 64),         # a single token
     (1, 2, 300, 64),       # 3 chunks, ragged tail; G = 1
     (1, 1, 129, 16),       # a full chunk + 1 token, 16 features (padded angles)
-    (2, 3, 1000, 256),     # 8 chunks; trig G = 4, ReLU G = 2
-    (1, 4, 127, 128),      # one ragged chunk; trig G = 2, ReLU G = 1
-    (1, 1, 400, 192),      # trig: 3 blocks round up to G = 4 with a padded block
+    (2, 3, 1000, 256),     # 8 chunks; G = 4
+    (1, 4, 127, 128),      # one ragged chunk; G = 2
+    (1, 1, 400, 192),      # 3 blocks round up to G = 4 with a padded block
 ])
 def test_causal_small(kind, B, H, L, M):
     c = Case(B, H, L, 64, M, seed=B * 100 + L + M + 7)
@@ -40,7 +40,7 @@ def test_causal_small(kind, B, H, L, M):
 
 
 def test_causal_relu_512_features():
-    # ReLU M = 512: G = 4 CTAs of 128 features
+    # ReLU M = 512: G = 8 CTAs of 64 features (16-row ownership blocks, one per CTA)
     c = Case(1, 2, 640, 64, 512, seed=11)
     g = _run(c, 1).reshape(2, 640, 64)
     ref, cond, _ = c.oracle(1, True)
@@ -48,7 +48,7 @@ def test_causal_relu_512_features():
 
 
 def test_causal_relu_384_features():
-    # ReLU M = 384: 128-angle blocks, 3 rounded up to G = 4 (one block is all padding)
+    # ReLU M = 384: 6 blocks of 64 angles rounded up to G = 8 (two blocks are all padding)
     c = Case(1, 2, 300, 64, 384, seed=12)
     g = _run(c, 1).reshape(2, 300, 64)
     ref, cond, _ = c.oracle(1, True)
@@ -150,3 +150,14 @@ def test_causal_chunk_argument():
     with pytest.raises(F.FavorError) as e:
         F.favor_attention(q, k, v, om, feature_kind=0, causal=True, chunk=64)
     assert e.value.code == -5
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+@pytest.mark.parametrize("d,M", [(16, 32), (32, 96), (16, 256)])
+def test_causal_head_sizes(kind, d, M):
+    # head sizes 16 and 32 ride in the 64-column boxes: zeros past d, d values stored per row
+    B, H, L = 2, 2, 600
+    c = Case(B, H, L, d, M, seed=d * 5 + M)
+    g = _run(c, kind).reshape(B * H, L, d)
+    ref, cond, _ = c.oracle(kind, True)
+    check_rows(g, ref, cond, TOL_BF16, U_BF16, f"causal d={d} M={M} kind={kind}", trig=kind == 0)
