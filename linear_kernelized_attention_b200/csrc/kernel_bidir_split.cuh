@@ -49,9 +49,9 @@ constexpr float kMargin = 16.f;     // stabiliser head-room above the largest |k
 constexpr int kThreads = 512;
 
 // Angles of 8 consecutive ones evaluated on the FMA pipe (bit j set: angle j of the group);
-// the rest go to the SFU. 0x49 = 3 of 8.
+// the rest go to the SFU. 0x00 (all on the SFU) measured fastest here: the kernels are bound by MMA issue and latency, not the SFU.
 #ifndef FAVOR_POLY_MASK
-#define FAVOR_POLY_MASK 0x49u
+#define FAVOR_POLY_MASK 0x00u
 #endif
 constexpr uint32_t kPolyMask = FAVOR_POLY_MASK;
 
@@ -60,6 +60,26 @@ __host__ __device__ inline long long run_begin(long long i, long long U, long lo
 __host__ __device__ inline long long cta_of_unit(long long x, long long U, long long P) {
   return ((x + 1) * P - 1) / U;
 }
+
+// Position of a tile in a CTA's run: the run starts tt0 tiles into its first pair (or head); the
+// walker advances tile by tile with no division, so the issuing warps never evaluate 64-bit
+// quotients in their loops.
+struct RunWalker {
+  int t, k, tt;   // tile of the run, pair (head) index within the run, tile within that pair
+  int n, nt;      // tiles in the run, tiles per pair
+  __device__ __forceinline__ RunWalker(int tt0, int n_, int nt_) : t(0), k(0), tt(tt0), n(n_), nt(nt_) {}
+  __device__ __forceinline__ void advance_to(int t_new) {
+    while (t < t_new) {
+      ++t;
+      if (++tt == nt) {
+        tt = 0;
+        ++k;
+      }
+    }
+  }
+  __device__ __forceinline__ bool first() const { return t == 0 || tt == 0; }
+  __device__ __forceinline__ bool last() const { return t == n - 1 || tt == nt - 1; }
+};
 
 // ============================================================================ key states
 template <int KIND, int DP>
@@ -124,9 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n = (int)(u1 - u0);  // tiles of this CTA
   const int nt = p.ntiles;
   const long long p0 = u0 / nt;  // first pair of the run
-  auto pair_of = [&](int t) { return (u0 + t) / nt; };
-  auto first_of_pair = [&](int t) { return t == 0 || (u0 + t) % nt == 0; };
-  auto last_of_pair = [&](int t) { return t == n - 1 || (u0 + t) % nt == nt - 1; };
+  const int tt0 = (int)(u0 - p0 * nt);
   auto slot_of = [&](long long pr) {
     return pr * p.smax + (blockIdx.x - cta_of_unit(pr * nt, U, P));
   };
@@ -187,11 +205,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tm_om);
       }
       int issued = 0, pk_issued = 0;
+      RunWalker w(tt0, n, nt);
+      int bh = 0, ab = 0, h = 0;
       for (int t = 0; t < n; ++t) {
-        const long long x = u0 + t, pr = x / nt;
-        const int pk = (int)(pr - p0);
-        const int bh = (int)(pr / p.nab), ab = (int)(pr % p.nab), h = bh % p.H;
-        if (first_of_pair(t)) {
+        w.advance_to(t);
+        const int pk = w.k;
+        if (w.first()) {
+          const int pr = (int)(p0 + pk);
+          bh = pr / p.nab;
+          ab = pr - bh * p.nab;
+          h = bh % p.H;
           if (pk >= 2 && !mbar_wait(bar(ms->om_free[pk & 1]), ((pk >> 1) - 1) & 1, abort_flag)) break;
           if (leader) {
             mbar_arrive_expect_tx(bar(ms->om_full[pk & 1]), C::kOmB);
@@ -204,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = t % NS;
         if (t >= NS && !mbar_wait(bar(ms->kv_empty[s]), ((t / NS) - 1) & 1, abort_flag)) break;
         const uint32_t st = s_stage + s * C::kStageB;
-        const int row = (int)(x % nt) * kTile;
+        const int row = w.tt * kTile;
         if (leader) {
           mbar_arrive_expect_tx(bar(ms->kv_full[s]), 2 * NCB * kBoxB);
           for (int kb = 0; kb < NCB; ++kb) {
@@ -232,11 +255,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t id2 = idesc_f16(128, NV, 1, 1, 0, 1);
       const int nitems = 2 * n;
       bool ok = true;
+      RunWalker w1(tt0, n, nt), w2(tt0, n, nt);  // the projection stream and the state stream
       auto mma1 = [&](int it) -> bool {
         const int t = it >> 1, hf = it & 1, s = t % NS, b = it % NBUF;
-        const int pk = (int)(pair_of(t) - p0);
+        w1.advance_to(t);
+        const int pk = w1.k;
         if (hf == 0) {
-          if (first_of_pair(t) && !mbar_wait(bar(ms->om_full[pk & 1]), (pk >> 1) & 1, abort_flag)) return false;
+          if (w1.first() && !mbar_wait(bar(ms->om_full[pk & 1]), (pk >> 1) & 1, abort_flag)) return false;
           if (!mbar_wait(bar(ms->kv_full[s]), (t / NS) & 1, abort_flag)) return false;
         }
         tc_fence_after();
@@ -252,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_ss(d, a0 + off, b0 + off, id1, (kb | kk) ? 1u : 0u);
             }
           mma_commit(bar(ms->u_full[b]));
-          if (hf == 1 && last_of_pair(t)) mma_commit(bar(ms->om_free[pk & 1]));
+          if (hf == 1 && w1.last()) mma_commit(bar(ms->om_free[pk & 1]));
         }
         __syncwarp();
         return true;
@@ -266,11 +291,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (KIND == 1) p.meta[sl * 2] = 0.f;
         }
       };
-      for (int it = 0; ok && it < NBUF && it < nitems; ++it) ok = mma1(it);
+      // projections run NBUF - 1 items ahead: the projection issued after item it's state product
+      // goes to the buffer item it - 1 used, whose product has long completed, so the tensor pipe
+      // gets both back to back and never drains waiting on the product just issued
+      for (int it = 0; ok && it < NBUF - 1 && it < nitems; ++it) ok = mma1(it);
       for (int it = 0; ok && it < nitems; ++it) {
         const int t = it >> 1, hf = it & 1, s = t % NS, b = it % NBUF;
-        const int pk = (int)(pair_of(t) - p0);
-        const bool fresh = hf == 0 && first_of_pair(t);
+        w2.advance_to(t);
+        const int pk = w2.k;
+        const bool fresh = hf == 0 && w2.first();
         if (!(ok = mbar_wait(bar(ms->p_full[b]), (it / NBUF) & 1, abort_flag))) break;
         if (KIND == 0 && hf == 0 && !(ok = mbar_wait(bar(ms->w_full[s]), (t / NS) & 1, abort_flag))) break;
         if (fresh && pk > 0) {
@@ -293,18 +322,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(bar(ms->buf_free[b]));
           if (hf == 1) {
             mma_commit(bar(ms->kv_empty[s]));
-            if (last_of_pair(t)) mma_commit(bar(ms->s_done));
+            if (w2.last()) mma_commit(bar(ms->s_done));
           }
         }
         __syncwarp();
-        const int nx = it + NBUF;
+        const int nx = it + NBUF - 1;
         if (nx < nitems) {
-          if (!(ok = mbar_wait(bar(ms->buf_free[b]), (it / NBUF) & 1, abort_flag))) break;
+          if (it >= 1 && !(ok = mbar_wait(bar(ms->buf_free[(it - 1) % NBUF]), ((it - 1) / NBUF) & 1, abort_flag)))
+            break;
           if (!(ok = mma1(nx))) break;
         }
       }
       if (ok) {
-        const int pk_last = (int)(pair_of(n - 1) - p0);
+        w2.advance_to(n - 1);
+        const int pk_last = w2.k;
         if (mbar_wait(bar(ms->s_free), pk_last & 1, abort_flag)) write_meta_max(pk_last);
       }
       if (leader) mma_commit(bar(ms->drain));
@@ -318,8 +349,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int j = (warp - 4) * 32 + lane;  // key row of the tile
       float c = 0.f;
       uint32_t nph = 0;
+      RunWalker rw(tt0, n, nt);
       for (int t = 0; t < n; ++t) {
-        const long long x = u0 + t;
+        rw.advance_to(t);
         const int s = t % NS;
         if (!mbar_wait(bar(ms->kv_full[s]), (t / NS) & 1, abort_flag)) break;
         uint8_t* st = gb + (s_stage - base) + s * C::kStageB;
@@ -338,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               acc = fmaf(hi, hi, acc);
             }
           }
-        const bool valid = (int)(x % nt) * kTile + j < p.L;
+        const bool valid = rw.tt * kTile + j < p.L;
         const float n2 = valid ? 0.5f * acc : -INFINITY;
         float m = n2;
 #pragma unroll
@@ -347,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!group_sync(bar(ms->norm_sync), nph, abort_flag)) break;
         m = fmaxf(fmaxf(ms->tmax[t & 1][0], ms->tmax[t & 1][1]), fmaxf(ms->tmax[t & 1][2], ms->tmax[t & 1][3]));
         float f = 1.f;
-        if (first_of_pair(t)) {
+        if (rw.first()) {
           c = m + kMargin;
         } else if (m > c) {
           const float cn = m + kMargin;
@@ -371,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<__nv_bfloat16*>(st + NCB * kBoxB + j * kRowB + ((j & 7) << 4)) = __float2bfloat16_rn(w);
         if (j == 0) {
           ms->frescale[s] = f;
-          if (last_of_pair(t)) p.meta[slot_of(x / nt) * 2] = c;
+          if (rw.last()) p.meta[slot_of(p0 + rw.k) * 2] = c;
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -384,10 +416,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t la = uint32_t(q * 32) << 16;
     const int nitems = 2 * n;
     bool ok = true;
+    RunWalker w(tt0, n, nt);
     for (int it = g; ok && it < nitems; it += 2) {
       const int t = it >> 1, hf = it & 1, s = t % NS, b = it % NBUF;
+      w.advance_to(t);
       if (!(ok = mbar_wait(bar(ms->u_full[b]), (it / NBUF) & 1, abort_flag))) break;
-      if (KIND == 0 && hf == 0 && !first_of_pair(t)) {
+      if (KIND == 0 && hf == 0 && !w.first()) {
         // the tile raised the reference: rescale S once every earlier state MMA has completed
         if (!(ok = mbar_wait(bar(ms->w_full[s]), (t / NS) & 1, abort_flag))) break;
         const float f = ms->frescale[s];
@@ -441,10 +475,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(ms->p_full[b]));
-      if (last_of_pair(t)) {
+      if (w.last()) {
         // flush: this group's share of the state to the pair's workspace slot
-        const long long pr = pair_of(t);
-        const int pk = (int)(pr - p0);
+        const int pk = w.k;
+        const long long pr = p0 + pk;
         if (!(ok = mbar_wait(bar(ms->s_done), pk & 1, abort_flag))) break;
         tc_fence_after();
         float* dst = p.part + slot_of(pr) * (long long)(DP + 1) * R;
@@ -593,9 +627,10 @@ template <int KIND, int DP>
 struct QueryCfg {
   static constexpr int NCB = DP / 64, NV = DP + 16;
   static constexpr int FB = KIND == 0 ? 256 : 128;   // features of a 128-angle block
-  static constexpr int NBN = DP == 64 ? 2 : 1;       // numerator buffers
+  static constexpr int NBQ = DP == 64 ? 3 : 2;       // 128-angle U/phi buffers
+  static constexpr int NBN = 1;                      // numerator buffers
   static constexpr int NOS = DP == 64 ? 2 : 1;       // output staging buffers
-  static constexpr int kNumCol = 256;                // TMEM: U ring [0, 256), numerators after
+  static constexpr int kNumCol = NBQ * 128;          // TMEM: U ring, then the numerator
   static_assert(kNumCol + NBN * NV <= 512, "TMEM budget");
 };
 
@@ -613,7 +648,7 @@ struct alignas(16) QueryMisc {
   uint32_t tmem_base;
   uint64_t head_full, head_free;
   uint64_t q_full[2], q_empty[2];
-  uint64_t u_full[2], p_full[2], buf_free[2];
+  uint64_t u_full[3], p_full[3], buf_free[3];
   uint64_t num_full[2], num_empty[2];
   uint64_t drain;
   uint64_t out_sync;  // bounded barrier among the 128 output threads
@@ -624,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_bidir_query(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_om,
                   const __grid_constant__ CUtensorMap tm_out, const QueryParams p) {
   using C = QueryCfg<KIND, DP>;
-  constexpr int NCB = C::NCB, NV = C::NV, FB = C::FB, NBN = C::NBN, NOS = C::NOS;
+  constexpr int NCB = C::NCB, NV = C::NV, FB = C::FB, NBN = C::NBN, NOS = C::NOS, NBQ = C::NBQ;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -640,9 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n = (int)(u1 - u0);
   const int nt = p.ntiles, nab = p.nab;
   const long long h0 = u0 / nt;
-  auto head_of = [&](int t) { return (u0 + t) / nt; };
-  auto first_of_head = [&](int t) { return t == 0 || (u0 + t) % nt == 0; };
-  auto last_of_head = [&](int t) { return t == n - 1 || (u0 + t) % nt == nt - 1; };
+  const int tt0 = (int)(u0 - h0 * nt);
 
   if (tid == 0) {
     ms->abort_flag = 0;
@@ -651,11 +684,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(ms->q_full[i]), 1);
       mbar_init(bar(ms->q_empty[i]), 1);
+      mbar_init(bar(ms->num_full[i]), 1);
+      mbar_init(bar(ms->num_empty[i]), 4);
+    }
+    for (int i = 0; i < 3; ++i) {
       mbar_init(bar(ms->u_full[i]), 1);
       mbar_init(bar(ms->p_full[i]), 8);
       mbar_init(bar(ms->buf_free[i]), 1);
-      mbar_init(bar(ms->num_full[i]), 1);
-      mbar_init(bar(ms->num_empty[i]), 4);
     }
     mbar_init(bar(ms->drain), 1);
     mbar_init(bar(ms->out_sync), 128);
@@ -681,19 +716,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tm_out);
       }
       int issued = 0, heads = 0;
+      RunWalker w(tt0, n, nt);
       for (int t = 0; t < n; ++t) {
-        const long long x = u0 + t, bh = x / nt;
+        w.advance_to(t);
+        const long long bh = h0 + w.k;
         const int s = t & 1;
         if (t >= 2 && !mbar_wait(bar(ms->q_empty[s]), ((t >> 1) - 1) & 1, abort_flag)) break;
         if (leader) {
           mbar_arrive_expect_tx(bar(ms->q_full[s]), NCB * kBoxB);
           for (int kb = 0; kb < NCB; ++kb)
-            tma_load_3d(s_q + (s * NCB + kb) * kBoxB, &tm_q, bar(ms->q_full[s]), kb * 64, (int)(x % nt) * kTile,
-                        (int)bh);
+            tma_load_3d(s_q + (s * NCB + kb) * kBoxB, &tm_q, bar(ms->q_full[s]), kb * 64, w.tt * kTile, (int)bh);
         }
         issued = t + 1;
-        if (first_of_head(t)) {
-          const int hk = (int)(bh - h0);
+        if (w.first()) {
+          const int hk = w.k;
           if (hk == 0) pdl_wait();  // the merge has written the state images
           if (hk >= 1 && !mbar_wait(bar(ms->head_free), (hk - 1) & 1, abort_flag)) break;
           const int h = (int)(bh % p.H);
@@ -731,14 +767,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t om0 = sdesc_sw128(s_om, 16, 1024);
       const uint64_t img0 = sdesc_sw128(s_img, 16, 1024);
       bool ok = true;
+      RunWalker w1(tt0, n, nt), w2(tt0, n, nt), w3(tt0, n, nt);  // projections, state products, look-ahead
       auto mma1 = [&](int j) -> bool {
-        const int t = j / nab, ab = j % nab, b = j & 1, s = t & 1;
+        const int t = j / nab, ab = j - t * nab, b = j % NBQ, s = t & 1;
+        w1.advance_to(t);
         if (ab == 0) {
           if (!mbar_wait(bar(ms->q_full[s]), (t >> 1) & 1, abort_flag)) return false;
-          if (first_of_head(t) && !mbar_wait(bar(ms->head_full), (int)(head_of(t) - h0) & 1, abort_flag))
-            return false;
+          if (w1.first() && !mbar_wait(bar(ms->head_full), w1.k & 1, abort_flag)) return false;
         }
-        if (j >= 2 && !mbar_wait(bar(ms->buf_free[b]), ((j - 2) >> 1) & 1, abort_flag)) return false;
+        if (j >= NBQ && !mbar_wait(bar(ms->buf_free[b]), ((j - NBQ) / NBQ) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint64_t q0 = sdesc_sw128(s_q + s * NCB * kBoxB, 16, 1024);
         if (leader) {
@@ -755,14 +792,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       int nx = 0;  // next item whose projection is to be issued
-      while (ok && nx < nit && nx < 2 && head_of(nx / nab) == h0) ok = mma1(nx++);
+      // projections run NBQ - 1 items ahead, into buffers whose products completed an item earlier
+      while (ok && nx < nit && nx < NBQ - 1) {
+        w3.advance_to(nx / nab);
+        if (w3.k != 0) break;
+        ok = mma1(nx++);
+      }
       for (int j = 0; ok && j < nit; ++j) {
-        const int t = j / nab, ab = j % nab, b = j & 1, nb = t % NBN;
-        if (!(ok = mbar_wait(bar(ms->p_full[b]), (j >> 1) & 1, abort_flag))) break;
+        const int t = j / nab, ab = j - t * nab, b = j % NBQ, nb = t % NBN;
+        w2.advance_to(t);
+        if (!(ok = mbar_wait(bar(ms->p_full[b]), (j / NBQ) & 1, abort_flag))) break;
         if (ab == 0 && t >= NBN && !(ok = mbar_wait(bar(ms->num_empty[nb]), ((t / NBN) - 1) & 1, abort_flag))) break;
         tc_fence_after();
         const uint32_t dn = tmem + C::kNumCol + nb * NV;
-        const bool head_end = ab == nab - 1 && last_of_head(t);
+        const bool head_end = ab == nab - 1 && w2.last();
         if (leader) {
 #pragma unroll
           for (int kk = 0; kk < FB / 16; ++kk) {
@@ -778,8 +821,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         // projections ahead: two items in flight, and none past a head change until the head's
         // last state product has been issued (the next head's Omega and image replace these)
-        while (ok && nx < nit && nx <= j + 2) {
-          const long long hn = head_of(nx / nab), hc = head_of(t);
+        while (ok && nx < nit && nx <= j + NBQ - 1) {
+          w3.advance_to(nx / nab);
+          const int hn = w3.k, hc = w2.k;
           if (!(hn == hc || (head_end && hn == hc + 1))) break;
           ok = mma1(nx++);
         }
@@ -795,7 +839,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t la = uint32_t(q * 32) << 16;
     const bool issuer = warp == 4 && lane == 0;
     uint32_t oph = 0;
+    RunWalker w(tt0, n, nt);
     for (int t = 0; t < n; ++t) {
+      w.advance_to(t);
       const int nb = t % NBN, sb = t % NOS;
       if (!mbar_wait(bar(ms->num_full[nb]), (t / NBN) & 1, abort_flag)) break;
       tc_fence_after();
@@ -835,9 +881,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       if (!group_sync(bar(ms->out_sync), oph, abort_flag)) break;
       if (issuer) {
-        const long long x = u0 + t;
         for (int kb = 0; kb < NCB; ++kb)
-          tma_store_3d(&tm_out, s_out + (sb * NCB + kb) * kBoxB, kb * 64, (int)(x % nt) * kTile, (int)(x / nt));
+          tma_store_3d(&tm_out, s_out + (sb * NCB + kb) * kBoxB, kb * 64, w.tt * kTile, (int)(h0 + w.k));
         bulk_commit();
       }
     }
@@ -848,8 +893,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t la = uint32_t(q * 32) << 16;
     const int nit = n * nab;
     for (int j = 0; j < nit; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait(bar(ms->u_full[b]), (j >> 1) & 1, abort_flag)) break;
+      const int b = j % NBQ;
+      if (!mbar_wait(bar(ms->u_full[b]), (j / NBQ) & 1, abort_flag)) break;
       tc_fence_after();
       const uint32_t ub = tmem + la + b * 128 + 64 * hcol;
 #pragma unroll 1

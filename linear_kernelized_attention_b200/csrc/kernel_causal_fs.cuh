@@ -61,7 +61,7 @@ constexpr int kRowB = 128;
 constexpr int kTileB = kTile * kRowB;  // 16 KB
 constexpr int kThreads = 544;
 #ifndef FAVOR_POLY_MASK_CAUSAL
-#define FAVOR_POLY_MASK_CAUSAL 0x49u
+#define FAVOR_POLY_MASK_CAUSAL 0x00u
 #endif
 constexpr uint32_t kPolyMask = FAVOR_POLY_MASK_CAUSAL;
 // Shared memory (offsets from the 1024-aligned base).
