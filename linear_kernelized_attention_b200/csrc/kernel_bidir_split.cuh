@@ -89,7 +89,7 @@ struct StateCfg {
   static constexpr int NSB = KIND == 0 ? 2 : 1;              // 128-row state blocks (trig: cos, sin)
   static constexpr int R = 128 * NSB;                        // state rows of a pair
   static constexpr int NBUF = (KIND == 0 && DP == 128) ? 3 : 4;  // 64-key U/phi buffers
-  static constexpr int NS = DP == 64 ? 3 : 2;                // K/V stages
+  static constexpr int NS = DP == 64 ? 4 : 2;                // K/V stages
   static constexpr int kStageB = (2 * NCB + 1) * kBoxB;      // V boxes | column box | K boxes
   static constexpr int kOmB = NCB * kBoxB;                   // one Omega block
   static constexpr int kUcol = (NSB * NV + 31) / 32 * 32;    // TMEM column of the U ring
@@ -113,10 +113,10 @@ struct alignas(16) StateMisc {
   int abort_flag;
   uint32_t tmem_base;
   float tmax[2][4];
-  float frescale[4];
+  float frescale[4];  // by stage
   float redmax[2][8];
   uint64_t om_full[2], om_free[2];
-  uint64_t kv_full[3], kv_empty[3], w_full[3];
+  uint64_t kv_full[4], kv_empty[4], w_full[4];
   uint64_t u_full[4], p_full[4], buf_free[4];
   uint64_t s_done, s_free, drain;
   uint64_t norm_sync;  // bounded barrier among the 128 norm threads
@@ -597,28 +597,55 @@ __global__ void __launch_bounds__(256) k_bidir_merge(const MergeParams p) {
   const int ns = min(nslots(pr, p), kMergeMaxSlots);
   uint8_t* img = p.img + bh * p.img_bytes;
   const float* part = p.part + pr * p.smax * (long long)(DP + 1) * R;
-  for (int e = threadIdx.x; e < 32 * NV; e += blockDim.x) {
-    const int rl = e & 31, nn = e >> 5;
-    const int r = rb * 32 + rl;
-    float v = 0.f;
+  const long long sstride = (long long)(DP + 1) * R;
+  // one work item = 8 consecutive state rows of one value row: two float4 loads per slot, and 8
+  // consecutive features of the image, i.e. one 16-byte chunk
+  for (int w = threadIdx.x; w < 4 * NV; w += blockDim.x) {
+    const int oct = w & 3, nn = w >> 2;
+    const int r0 = rb * 32 + oct * 8;
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (nn <= DP) {
-      const float* src = part + (long long)nn * R + r;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const float* src = part + (long long)nn * R + r0;
       int s = 0;
-      for (; s + 4 <= ns; s += 4) {
-#pragma unroll
-        for (int t = 0; t < 4; ++t) acc[t] = fmaf(wts[s + t], src[(long long)(s + t) * (DP + 1) * R], acc[t]);
+      for (; s + 2 <= ns; s += 2) {
+        const float4 a0 = *reinterpret_cast<const float4*>(src + s * sstride);
+        const float4 a1 = *reinterpret_cast<const float4*>(src + s * sstride + 4);
+        const float4 b0 = *reinterpret_cast<const float4*>(src + (s + 1) * sstride);
+        const float4 b1 = *reinterpret_cast<const float4*>(src + (s + 1) * sstride + 4);
+        const float wa = wts[s], wb = wts[s + 1];
+        v[0] = fmaf(wa, a0.x, fmaf(wb, b0.x, v[0]));
+        v[1] = fmaf(wa, a0.y, fmaf(wb, b0.y, v[1]));
+        v[2] = fmaf(wa, a0.z, fmaf(wb, b0.z, v[2]));
+        v[3] = fmaf(wa, a0.w, fmaf(wb, b0.w, v[3]));
+        v[4] = fmaf(wa, a1.x, fmaf(wb, b1.x, v[4]));
+        v[5] = fmaf(wa, a1.y, fmaf(wb, b1.y, v[5]));
+        v[6] = fmaf(wa, a1.z, fmaf(wb, b1.z, v[6]));
+        v[7] = fmaf(wa, a1.w, fmaf(wb, b1.w, v[7]));
       }
-      for (; s < ns; ++s) acc[0] = fmaf(wts[s], src[(long long)s * (DP + 1) * R], acc[0]);
-      v = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      if (s < ns) {
+        const float4 a0 = *reinterpret_cast<const float4*>(src + s * sstride);
+        const float4 a1 = *reinterpret_cast<const float4*>(src + s * sstride + 4);
+        const float wa = wts[s];
+        v[0] = fmaf(wa, a0.x, v[0]);
+        v[1] = fmaf(wa, a0.y, v[1]);
+        v[2] = fmaf(wa, a0.z, v[2]);
+        v[3] = fmaf(wa, a0.w, v[3]);
+        v[4] = fmaf(wa, a1.x, v[4]);
+        v[5] = fmaf(wa, a1.y, v[5]);
+        v[6] = fmaf(wa, a1.z, v[6]);
+        v[7] = fmaf(wa, a1.w, v[7]);
+      }
     }
-    const int a = KIND == 0 ? (r & 127) : r;
-    if (ab * 128 + a >= p.M) v = 0.f;  // padded angle
-    const int f = KIND == 0 ? ab * FB + (a >> 5) * 64 + (r >> 7) * 32 + (a & 31) : ab * FB + r;
-    if (KIND == 0)
-      *reinterpret_cast<__half*>(img + img_byte<NV>(f, nn)) = __float2half_rn(v * scale);
-    else
-      *reinterpret_cast<__nv_bfloat16*>(img + img_byte<NV>(f, nn)) = __float2bfloat16_rn(v);
+    const int a0 = KIND == 0 ? (r0 & 127) : r0;  // first angle of the octet (same sin/cos block)
+    uint32_t pk[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float x0 = ab * 128 + a0 + 2 * e < p.M ? v[2 * e] : 0.f;      // padded angles read as zero
+      const float x1 = ab * 128 + a0 + 2 * e + 1 < p.M ? v[2 * e + 1] : 0.f;
+      pk[e] = KIND == 0 ? pack_f16x2(x0 * scale, x1 * scale) : pack_bf16x2(x0, x1);
+    }
+    const int f0 = KIND == 0 ? ab * FB + (a0 >> 5) * 64 + (r0 >> 7) * 32 + (a0 & 31) : ab * FB + r0;
+    *reinterpret_cast<uint4*>(img + img_byte<NV>(f0, nn)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
   }
 }
 

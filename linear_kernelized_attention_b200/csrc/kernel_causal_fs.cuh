@@ -42,10 +42,11 @@
 //              phi(Q).z with z split into bf16 hi and lo rows, intra = P16 V_c
 // The intra denominator sum_j P16_ij is accumulated in fp32 registers.
 //
-// Warp roles (544 threads): 0 TMA; 1 TMEM allocator and issuer A; 2 issuer B; 3 key norms and
-// references; 4-7 state image and phi'(K) (thread = feature / key row); 8-11 phi(Q) (thread =
-// query row; two TMEM slots, so the next chunk's features overlap this chunk's products);
-// 12-15 P16 and partial rows (thread = query row); 16 combiner of the owned rows.
+// Warp roles (544 threads): 0 TMA; 1 TMEM allocator and issuer A (U_K(c + 1) is issued before
+// the state update of chunk c); 2 issuer B; 3 key norms and references; 4-7 phi'(K) (thread =
+// key row); 8-11 the state image, then phi(Q) (thread = feature row, then query row; two phi(Q)
+// slots, so the next chunk's features overlap this chunk's products); 12-15 P16 and partial rows
+// (thread = query row); 16 combiner of the owned rows.
 // Head sizes 16 and 32 ride in the 64-column boxes (zeros past d).
 #pragma once
 #include <cuda_bf16.h>
@@ -297,6 +298,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       bool ok = mbar_wait(bar(ms->om_full), 0, abort_flag) && (nch == 0 || uk(0));
       for (int c = 0; ok && c < nch; ++c) {
+        // U_K(c + 1) first: it needs only the next K tile and the phi(K) warps' copy of U_K(c), so
+        // their next chunk does not wait for this chunk's state image and update
+        if (c + 1 < nch && !(ok = uk(c + 1))) break;
         // S += phi(K)^T [w o V], z += phi(K)^T w
         if (!(ok = mbar_wait(bar(ms->phik_full[c & 1]), (c >> 1) & 1, abort_flag))) break;
         if (!(ok = mbar_wait(bar(ms->s_ready), c & 1, abort_flag))) break;
@@ -317,7 +321,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(bar(ms->v_empty[c & 1]));  // the V tile has been read
         }
         __syncwarp();
-        if (c + 1 < nch && !(ok = uk(c + 1))) break;
       }
       if (leader) mma_commit(bar(ms->drain_a));
       __syncwarp();
@@ -497,18 +500,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       crefl = cnewl;
     }
   } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ phi(K) and the state image
+    // ------------------------------------------------------------ phi(K)
     const int q4 = warp & 3, row = q4 * 32 + lane;
     const uint32_t la = uint32_t(q4 * 32) << 16;
-    // z_f as bf16 hi + lo parts in rows 0 and 1 of the K-major z operand (128-byte swizzle)
-    auto zrow_store = [&](float z) {
-      const __nv_bfloat16 hi = __float2bfloat16_rn(z);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(z - __bfloat162float(hi));
-      uint8_t* zb = gb + kC_ZROW + (row >> 6) * 2048 + (row & 7) * 2;
-      const int ch = (row & 63) >> 3;
-      *reinterpret_cast<__nv_bfloat16*>(zb + (ch << 4)) = hi;
-      *reinterpret_cast<__nv_bfloat16*>(zb + kRowB + ((ch ^ 1) << 4)) = lo;
-    };
     // phi'(K_c) = a_j phi(k_j) into buffer c & 1, once P(c-2) and S(c-2) have read that buffer
     // (S(c-2) is complete: the state image of chunk c-1 waited for it)
     auto phi_k = [&](int c) -> bool {
@@ -566,7 +560,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(bar(ms->phik_full[c & 1]));
       return true;
     };
-    bool ok = nch == 0 || phi_k(0);
+    for (int c = 0; c < nch; ++c)
+      if (!phi_k(c)) break;
+  } else if (warp < 12) {
+    // ------------------------------------------------------------ state image and phi(Q)
+    // (thread = feature row for the image, query row for phi(Q); two phi(Q) slots)
+    const int q4 = warp & 3, row = q4 * 32 + lane;
+    const uint32_t la = uint32_t(q4 * 32) << 16;
+    // z_f as bf16 hi + lo parts in rows 0 and 1 of the K-major z operand (128-byte swizzle)
+    auto zrow_store = [&](float z) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(z);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(z - __bfloat162float(hi));
+      uint8_t* zb = gb + kC_ZROW + (row >> 6) * 2048 + (row & 7) * 2;
+      const int ch = (row & 63) >> 3;
+      *reinterpret_cast<__nv_bfloat16*>(zb + (ch << 4)) = hi;
+      *reinterpret_cast<__nv_bfloat16*>(zb + kRowB + ((ch ^ 1) << 4)) = lo;
+    };
+    bool ok = true;
     for (int c = 0; ok && c < nch; ++c) {
       const int mb = c & (kMeta - 1);
       // image of S_{<c} at reference cref_c, then S rescaled to cnew_c
@@ -620,13 +630,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(ms->img_full));
         mbar_arrive(bar(ms->s_ready));
       }
-      if (c + 1 < nch && !(ok = phi_k(c + 1))) break;
-    }
-  } else if (warp < 12) {
-    // ------------------------------------------------------------ phi(Q), two slots
-    const int q4 = warp & 3;
-    const uint32_t la = uint32_t(q4 * 32) << 16;
-    for (int c = 0; c < nch; ++c) {
       const uint32_t slot = tmem + la + kT_A + (c & 1) * 64;
       if (!mbar_wait(bar(ms->uq_full[c & 1]), (c >> 1) & 1, abort_flag)) break;
       tc_fence_after();
