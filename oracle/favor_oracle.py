@@ -280,7 +280,7 @@ def row_diagnostics_head(q, k, v, Om, kind, causal, rows=None):
     return kappa, s
 
 
-def row_condition_head(q, k, v, Om, kind, causal, rows=None):
+def row_condition_head(q, k, v, Om, kind, causal, rows=None, with_den=False):
     """Relative condition number of each chosen output row under rounding of the features.
 
     The method computes out_i = sum_f phi_f(q_i) S_f / sum_f phi_f(q_i) z_f with
@@ -292,6 +292,13 @@ def row_condition_head(q, k, v, Om, kind, causal, rows=None):
         cond_i = (max|N_i| + max|out_i| D_i) / (|den_i| max|out_i|).
     The trig map cancels across features as well as keys, so cond_i can reach 1e5 where
     kappa_i is small. Causal sums run over j <= i.
+
+    with_den=True also returns kappa_i = D_i / |den_i|, the condition of the denominator alone.
+    Past first order the same perturbations give exactly
+        |d out_i| <= u (N_i + |out_i| D_i) / (|den_i| (1 - u kappa_i))   while u kappa_i < 1,
+    and once u kappa_i >= 1 they can cancel den_i altogether, so no bound holds: this is the
+    trig mode's occasional numerical instability that the explainer's engineering notes set
+    against the stable non-negative mode ([EXPL], the paragraph on the two feature modes).
     """
     L = q.shape[0]
     rows = np.arange(L) if rows is None else np.asarray(rows)
@@ -328,7 +335,68 @@ def row_condition_head(q, k, v, Om, kind, causal, rows=None):
     out = _normalise(num, den)
     on = np.abs(out).max(axis=1)
     with np.errstate(divide="ignore", invalid="ignore"):
-        return (np.abs(N).max(axis=1) + on * D) / (np.abs(den) * on)
+        cond = (np.abs(N).max(axis=1) + on * D) / (np.abs(den) * on)
+        if not with_den:
+            return cond
+        return cond, D / np.abs(den)
+
+
+def row_rounding_terms_head(q, k, v, Om, kind, causal, rows=None):
+    """Sums of squares of the terms that each rounding level of the linear-time form touches.
+
+    [EXPL, 核心机制] evaluates num_i = phi(q_i)^T S and den_i = phi(q_i)^T z with the state
+    S = sum_j phi(k_j) v_j^T, z = sum_j phi(k_j) (j <= i when causal). Rounding in a finite
+    precision enters at three levels; with independent relative errors e of mean zero and
+    variance s^2 at one level, the variance of num_in is s^2 times:
+      level 1, one error per (feature f, key j) (the key features):
+          N1_in = sum_f sum_j (phi_f(q_i) phi_f(k_j) v_jn)^2,   D1_i = sum_f sum_j (phi_f(q_i) phi_f(k_j))^2
+      level 2, one error per (query i, key j) or per (key j, column n) (values, masked products):
+          N2_in = sum_j (A_ij v_jn)^2,   D2_i = sum_j A_ij^2,   A_ij = phi(q_i)^T phi(k_j)
+      level 3, one error per (feature f, column n) (query features, the state):
+          N3_in = sum_f (phi_f(q_i) S_fn)^2,   D3_i = sum_f (phi_f(q_i) z_f)^2
+    Returns a dict of out [rows, dv], den [rows] and N1, N2, N3 [rows, dv], D1, D2, D3 [rows].
+    Nothing here depends on how a kernel blocks the sums; the tests combine the levels with
+    the unit roundoffs of a path's operand types (probabilistic rounding error analysis in the
+    sense of Higham and Mary, SIAM J. Sci. Comput. 41(5), 2019).
+    """
+    L = q.shape[0]
+    rows = np.arange(L) if rows is None else np.asarray(rows)
+    fq = phi(q[rows], Om, kind)
+    fk = phi(k, Om, kind)
+    A = fq @ fk.T
+    if causal:
+        A = np.where(np.arange(L)[None, :] <= rows[:, None], A, 0.0)
+    t = {"N2": (A * A) @ (v * v), "D2": (A * A).sum(axis=1)}
+    fq2, fk2, v2 = fq * fq, fk * fk, v * v
+    if not causal:
+        S, z = fk.T @ v, fk.sum(axis=0)
+        num, den = fq @ S, fq @ z
+        t["N1"], t["D1"] = fq2 @ (fk2.T @ v2), fq2 @ fk2.sum(axis=0)
+        t["N3"], t["D3"] = fq2 @ (S * S), fq2 @ (z * z)
+    else:
+        F, dv = fk.shape[1], v.shape[1]
+        n = len(rows)
+        num, den = np.zeros((n, dv)), np.zeros(n)
+        for key in ("N1", "N3"):
+            t[key] = np.zeros((n, dv))
+        for key in ("D1", "D3"):
+            t[key] = np.zeros(n)
+        S, z = np.zeros((F, dv)), np.zeros(F)
+        SS, zz = np.zeros((F, dv)), np.zeros(F)
+        j0 = 0                       # keys [0, j0) are in the prefix sums
+        for r in np.argsort(rows, kind="stable"):
+            j1 = rows[r] + 1
+            if j1 > j0:
+                S += fk[j0:j1].T @ v[j0:j1]
+                z += fk[j0:j1].sum(axis=0)
+                SS += fk2[j0:j1].T @ v2[j0:j1]
+                zz += fk2[j0:j1].sum(axis=0)
+                j0 = j1
+            num[r], den[r] = fq[r] @ S, fq[r] @ z
+            t["N1"][r], t["D1"][r] = fq2[r] @ SS, fq2[r] @ zz
+            t["N3"][r], t["D3"][r] = fq2[r] @ (S * S), fq2[r] @ (z * z)
+    t["out"], t["den"] = _normalise(num, den), den
+    return t
 
 
 def favor_rows_head(q, k, v, Om, kind, causal, rows):

@@ -5,6 +5,7 @@ import numpy as np
 
 import favor_inputs as fi
 from oracle import favor_oracle as O
+from parity_util import RowCond
 
 
 class Case:
@@ -24,9 +25,9 @@ class Case:
         return self._dev
 
     def oracle(self, kind, causal, heads=None, rows=None):
-        """Oracle rows [n_heads, n_rows, d] and their condition numbers [n_heads, n_rows]."""
+        """Oracle rows [n_heads, n_rows, d] and a RowCond of their condition numbers [n_heads, n_rows]."""
         heads = [(b, h) for b in range(self.B) for h in range(self.H)] if heads is None else heads
-        outs, conds = [], []
+        outs, conds, terms = [], [], []
         for b, h in heads:
             a = (self.q[b, h], self.k[b, h], self.v[b, h], self.om[h])
             r = np.arange(self.L) if rows is None else np.asarray(rows)
@@ -37,5 +38,9 @@ class Case:
             else:
                 o = O.favor_rows_head(*a, kind, causal, r)
             outs.append(o)
-            conds.append(O.row_condition_head(*a, kind, causal, r))
-        return np.stack(outs), np.stack(conds), heads
+            conds.append(O.row_condition_head(*a, kind, causal, r, with_den=True))
+            if kind == O.TRIG:
+                terms.append(O.row_rounding_terms_head(*a, kind, causal, r))
+        tm = {key: np.stack([t[key] for t in terms]) for key in terms[0]} if terms else None
+        return (np.stack(outs), RowCond(np.stack([c for c, _ in conds]), np.stack([k for _, k in conds]), tm),
+                heads)

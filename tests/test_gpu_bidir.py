@@ -8,7 +8,7 @@ import pytest
 
 import favor_inputs as fi
 from cases import Case
-from parity_util import TOL_BF16, U_BF16, check_rows
+from parity_util import TOL_BF16, U_BIDIR16, check_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -34,7 +34,7 @@ def test_bidir_small(kind, B, H, L, M):
     c = Case(B, H, L, 64, M, seed=B * 100 + L + M)
     g = _run(c, kind).reshape(B * H, L, 64)
     ref, cond, _ = c.oracle(kind, False)
-    check_rows(g, ref, cond, TOL_BF16, U_BF16, f"kind={kind} {B}x{H}x{L} M={M}", trig=kind == 0)
+    check_rows(g, ref, cond, TOL_BF16, U_BIDIR16, f"kind={kind} {B}x{H}x{L} M={M}", trig=kind == 0)
 
 
 @pytest.mark.parametrize("kind", [0, 1])
@@ -45,7 +45,7 @@ def test_bidir_many_heads_single_cta_per_head(kind):
     heads = [(0, 0), (0, 79), (1, 40), (1, 79)]
     ref, cond, _ = c.oracle(kind, False, heads=heads)
     sel = np.stack([g[b * 80 + h] for b, h in heads])
-    check_rows(sel, ref, cond, TOL_BF16, U_BF16, f"many heads kind={kind}", trig=kind == 0)
+    check_rows(sel, ref, cond, TOL_BF16, U_BIDIR16, f"many heads kind={kind}", trig=kind == 0)
 
 
 def test_bidir_protein_mlm_shape_trig():
@@ -53,7 +53,7 @@ def test_bidir_protein_mlm_shape_trig():
     c = Case(8, 8, 1024, 64, 256, seed=0)
     g = _run(c, 0).reshape(64, 1024, 64)
     ref, cond, _ = c.oracle(0, False)
-    st = check_rows(g, ref, cond, TOL_BF16, U_BF16, "B8 H8 L1024 trig")
+    st = check_rows(g, ref, cond, TOL_BF16, U_BIDIR16, "B8 H8 L1024 trig")
     print(st)
 
 
@@ -63,7 +63,7 @@ def test_bidir_bench_workload(kind):
     c = Case(4, 8, 4096, 64, 256, seed=0)
     g = _run(c, kind).reshape(32, 4096, 64)
     ref, cond, _ = c.oracle(kind, False)
-    st = check_rows(g, ref, cond, TOL_BF16, U_BF16, f"bench kind={kind}", trig=kind == 0)
+    st = check_rows(g, ref, cond, TOL_BF16, U_BIDIR16, f"bench kind={kind}", trig=kind == 0)
     print(st)
 
 
@@ -79,7 +79,7 @@ def test_bidir_stabiliser_rescale():
     c._dev = None
     g = _run(c, 0).reshape(1, 1024, 64)
     ref, cond, _ = c.oracle(0, False)
-    check_rows(g, ref, cond, TOL_BF16, U_BF16, "rescale")
+    check_rows(g, ref, cond, TOL_BF16, U_BIDIR16, "rescale")
 
 
 def test_bidir_constant_v_and_zero_queries():
@@ -95,7 +95,7 @@ def test_bidir_constant_v_and_zero_queries():
         # the exact answer is the constant row; trig rows with heavy cancellation get the
         # condition-aware allowance like every other parity check
         np.testing.assert_allclose(ref, np.broadcast_to(fi.as_f64(val), ref.shape), rtol=1e-9, atol=1e-9)
-        check_rows(g, ref, cond, TOL_BF16, U_BF16, f"constant v kind={kind}", trig=kind == 0)
+        check_rows(g, ref, cond, TOL_BF16, U_BIDIR16, f"constant v kind={kind}", trig=kind == 0)
     # ReLU with q = 0: every feature of q is 0, so the denominator is 0 and the row is 0
     c.t[0] = torch.zeros_like(c.t[0])
     c._dev = None
@@ -111,7 +111,7 @@ def test_bidir_long_sequence_sampled_rows():
     heads = [(0, 0), (0, 15)]
     ref, cond, _ = c.oracle(0, False, heads=heads, rows=rows)
     sel = np.stack([g[h][rows] for _, h in heads])
-    check_rows(sel, ref, cond, TOL_BF16, U_BF16, "L=65536 sampled")
+    check_rows(sel, ref, cond, TOL_BF16, U_BIDIR16, "L=65536 sampled")
 
 
 @pytest.mark.parametrize("kind", [0, 1])
@@ -123,7 +123,7 @@ def test_bidir_head_sizes(kind, d, M):
     c = Case(B, H, L, d, M, seed=d * 7 + M)
     g = _run(c, kind).reshape(B * H, L, d)
     ref, cond, _ = c.oracle(kind, False)
-    check_rows(g, ref, cond, TOL_BF16, U_BF16, f"d={d} M={M} kind={kind}", trig=kind == 0)
+    check_rows(g, ref, cond, TOL_BF16, U_BIDIR16, f"d={d} M={M} kind={kind}", trig=kind == 0)
 
 
 def test_bidir_unsupported_shapes_are_refused():

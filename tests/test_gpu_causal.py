@@ -10,7 +10,7 @@ import pytest
 
 import favor_inputs as fi
 from cases import Case
-from parity_util import TOL_BF16, U_BF16, check_rows
+from parity_util import TOL_BF16, U_CAUSAL16, check_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -36,7 +36,7 @@ def test_causal_small(kind, B, H, L, M):
     c = Case(B, H, L, 64, M, seed=B * 100 + L + M + 7)
     g = _run(c, kind).reshape(B * H, L, 64)
     ref, cond, _ = c.oracle(kind, True)
-    check_rows(g, ref, cond, TOL_BF16, U_BF16, f"causal kind={kind} {B}x{H}x{L} M={M}", trig=kind == 0)
+    check_rows(g, ref, cond, TOL_BF16, U_CAUSAL16, f"causal kind={kind} {B}x{H}x{L} M={M}", trig=kind == 0)
 
 
 def test_causal_relu_512_features():
@@ -44,7 +44,7 @@ def test_causal_relu_512_features():
     c = Case(1, 2, 640, 64, 512, seed=11)
     g = _run(c, 1).reshape(2, 640, 64)
     ref, cond, _ = c.oracle(1, True)
-    check_rows(g, ref, cond, TOL_BF16, U_BF16, "causal relu M=512", trig=False)
+    check_rows(g, ref, cond, TOL_BF16, U_CAUSAL16, "causal relu M=512", trig=False)
 
 
 def test_causal_relu_384_features():
@@ -52,7 +52,7 @@ def test_causal_relu_384_features():
     c = Case(1, 2, 300, 64, 384, seed=12)
     g = _run(c, 1).reshape(2, 300, 64)
     ref, cond, _ = c.oracle(1, True)
-    check_rows(g, ref, cond, TOL_BF16, U_BF16, "causal relu M=384", trig=False)
+    check_rows(g, ref, cond, TOL_BF16, U_CAUSAL16, "causal relu M=384", trig=False)
 
 
 @pytest.mark.parametrize("kind", [0, 1])
@@ -63,7 +63,7 @@ def test_causal_more_heads_than_sms(kind):
     heads = [(0, 0), (0, 79), (1, 40), (1, 79)]
     ref, cond, _ = c.oracle(kind, True, heads=heads)
     sel = np.stack([g[b * 80 + h] for b, h in heads])
-    check_rows(sel, ref, cond, TOL_BF16, U_BF16, f"causal many heads kind={kind}", trig=kind == 0)
+    check_rows(sel, ref, cond, TOL_BF16, U_CAUSAL16, f"causal many heads kind={kind}", trig=kind == 0)
 
 
 def test_causal_first_row_is_v0():
@@ -80,7 +80,7 @@ def test_causal_bench_workload(kind):
     c = Case(4, 8, 4096, 64, 256, seed=0)
     g = _run(c, kind).reshape(32, 4096, 64)
     ref, cond, _ = c.oracle(kind, True)
-    st = check_rows(g, ref, cond, TOL_BF16, U_BF16, f"causal bench kind={kind}", trig=kind == 0)
+    st = check_rows(g, ref, cond, TOL_BF16, U_CAUSAL16, f"causal bench kind={kind}", trig=kind == 0)
     print(st)
 
 
@@ -92,7 +92,7 @@ def test_causal_heavy_norm_decoder():
     heads = [(0, 0), (1, 7)]
     ref, cond, _ = c.oracle(0, True, heads=heads, rows=rows)
     sel = np.stack([g[b * 8 + h][rows] for b, h in heads])
-    st = check_rows(sel, ref, cond, TOL_BF16, U_BF16, "causal heavy-norm")
+    st = check_rows(sel, ref, cond, TOL_BF16, U_CAUSAL16, "causal heavy-norm")
     print(st)
 
 
@@ -109,7 +109,7 @@ def test_causal_key_norm_jump_inside_a_chunk():
     c._dev = None
     g = _run(c, 0).reshape(1, 1024, 64)
     ref, cond, _ = c.oracle(0, True)
-    check_rows(g, ref, cond, TOL_BF16, U_BF16, "causal norm jump")
+    check_rows(g, ref, cond, TOL_BF16, U_CAUSAL16, "causal norm jump")
 
 
 def test_causal_constant_v_and_zero_queries():
@@ -122,7 +122,7 @@ def test_causal_constant_v_and_zero_queries():
     for kind in (0, 1):
         g = _run(c, kind).reshape(2, 500, 64)
         ref, cond, _ = c.oracle(kind, True)
-        check_rows(g, ref, cond, TOL_BF16, U_BF16, f"causal constant v kind={kind}", trig=kind == 0)
+        check_rows(g, ref, cond, TOL_BF16, U_CAUSAL16, f"causal constant v kind={kind}", trig=kind == 0)
     # ReLU with q = 0: every query feature is 0, the denominator is 0 and the row is 0
     c.t[0] = torch.zeros_like(c.t[0])
     c._dev = None
@@ -137,7 +137,7 @@ def test_causal_long_sequence_sampled_rows():
     heads = [(0, 0), (0, 15)]
     ref, cond, _ = c.oracle(0, True, heads=heads, rows=rows)
     sel = np.stack([g[h][rows] for _, h in heads])
-    check_rows(sel, ref, cond, TOL_BF16, U_BF16, "causal L=65536 sampled")
+    check_rows(sel, ref, cond, TOL_BF16, U_CAUSAL16, "causal L=65536 sampled")
 
 
 def test_causal_chunk_argument():
@@ -160,4 +160,4 @@ def test_causal_head_sizes(kind, d, M):
     c = Case(B, H, L, d, M, seed=d * 5 + M)
     g = _run(c, kind).reshape(B * H, L, d)
     ref, cond, _ = c.oracle(kind, True)
-    check_rows(g, ref, cond, TOL_BF16, U_BF16, f"causal d={d} M={M} kind={kind}", trig=kind == 0)
+    check_rows(g, ref, cond, TOL_BF16, U_CAUSAL16, f"causal d={d} M={M} kind={kind}", trig=kind == 0)

@@ -15,7 +15,7 @@ import pytest
 import favor_inputs as fi
 from cases import Case
 from oracle import favor_oracle as O
-from parity_util import check_rows
+from parity_util import TOL_BF16, U_CAUSAL16, check_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -124,7 +124,7 @@ def test_decode_matches_tensor_core_causal_path():
         p = fi.as_f64(F.favor_attention(q, k, v, om, feature_kind=kind, causal=True)).reshape(8, 260, 64)
         ref, cond, _ = c.oracle(kind, True)
         check_rows(g, ref, cond, TOL_DEC, U_DEC, "decode", trig=kind == 0, headroom=1.0)
-        check_rows(p, ref, cond, 2e-2, 2.0 ** -8, "chunked", trig=kind == 0)
+        check_rows(p, ref, cond, TOL_BF16, U_CAUSAL16, "chunked", trig=kind == 0)
 
 
 def test_decode_zero_query_relu_and_reinit():

@@ -6,8 +6,9 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("d,M,kind,causal", [
-    (32, 64, 0, False), (32, 64, 1, True),        # d other than 64
-    (64, 40, 0, False), (64, 40, 1, True),        # M not a multiple of 16
+    (48, 64, 0, False), (48, 64, 1, True),        # d not 16, 32, 64 or 128
+    (128, 64, 0, True), (128, 64, 1, True),       # causal d = 128
+    (128, 256, 0, False),                         # trig d = 128 with M = 256: no shared-memory plan
     (64, 272, 0, False), (64, 272, 0, True),      # trig M > 256
     (64, 528, 1, False), (64, 528, 1, True),      # relu M > 512
 ])

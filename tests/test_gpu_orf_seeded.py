@@ -72,7 +72,7 @@ def test_seeded_omega_drives_attention():
     import torch
     import favor_inputs as fi
     import linear_kernelized_attention_b200 as F
-    from parity_util import TOL_BF16, U_BF16, check_rows
+    from parity_util import TOL_BF16, U_CAUSAL16, RowCond, check_rows
     B, H, L, d, M = 1, 2, 300, 64, 128
     om = F.favor_orf_omega_seeded(77, H, M, d, dtype=torch.bfloat16)
     q, k, v = (fi.round_to(x, "bf16") for x in fi.qkv(B, H, L, d, seed=3))
@@ -80,5 +80,9 @@ def test_seeded_omega_drives_attention():
     Q, K, V, OM = fi.as_f64(q), fi.as_f64(k), fi.as_f64(v), fi.as_f64(om.cpu())
     for h in range(H):
         ref = O.favor_causal_head(Q[0, h], K[0, h], V[0, h], OM[h], O.TRIG)
-        cond = O.row_condition_head(Q[0, h], K[0, h], V[0, h], OM[h], O.TRIG, True)
-        check_rows(fi.as_f64(out[0, h].cpu())[None], ref[None], cond[None], TOL_BF16, U_BF16, "seeded omega")
+        a = (Q[0, h], K[0, h], V[0, h], OM[h], O.TRIG, True)
+        cond, kden = O.row_condition_head(*a, with_den=True)
+        t = O.row_rounding_terms_head(*a)
+        check_rows(fi.as_f64(out[0, h].cpu())[None], ref[None],
+                   RowCond(cond[None], kden[None], {key: x[None] for key, x in t.items()}),
+                   TOL_BF16, U_CAUSAL16, "seeded omega")

@@ -542,3 +542,121 @@ def test_row_condition_bounds_feature_perturbations(kind, causal):
     if kind == O.RELU:
         # all terms non-negative: D_i = den_i, so cond_i = N_i/(den_i |o_i|) + 1 is modest
         assert cond.max() < 1e3
+
+
+def _terms(q, k, om, kind, causal):
+    """Products t[i, f, j] = phi_f(q_i) phi_f(k_j), zero where j > i when causal."""
+    fq, fk = O.phi(q, om, kind), O.phi(k, om, kind)
+    t = fq[:, :, None] * fk.T[None, :, :]
+    if causal:
+        t = t * (np.arange(k.shape[0])[None, None, :] <= np.arange(q.shape[0])[:, None, None])
+    return t
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_denominator_condition_is_attained(causal):
+    # every product moved by u |t| against the sign of den_i moves den_i by exactly u D_i: at
+    # u = 0.999 / kappa_i the denominator keeps its sign with |den_i| (1 - u kappa_i) left, at
+    # u = 1.001 / kappa_i it changes sign. This fixes both D_i and |den_i|.
+    q, k, v = _qkv(80, 16, seed=52)
+    om = _orf(32, 16, seed=52)[0]
+    _, kden = O.row_condition_head(q, k, v, om, O.TRIG, causal, with_den=True)
+    t = _terms(q, k, om, O.TRIG, causal)
+    den = t.sum(axis=(1, 2))
+    sgn = np.sign(den)[:, None, None]
+    for frac in (0.999, 1.001):
+        u = (frac / kden)[:, None, None]
+        den2 = (t - u * np.abs(t) * sgn).sum(axis=(1, 2))
+        if frac < 1:
+            assert np.all(np.sign(den2) == np.sign(den))
+            np.testing.assert_allclose(np.abs(den2), np.abs(den) * (1 - frac), rtol=1e-6)
+        else:
+            assert np.all(np.sign(den2) == -np.sign(den))
+    # ReLU products are non-negative: the denominator is perfectly conditioned
+    _, kr = O.row_condition_head(q, k, v, om, O.RELU, causal, with_den=True)
+    ok = np.isfinite(kr)
+    np.testing.assert_allclose(kr[ok], 1.0, rtol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_all_orders_bound_holds_far_from_first_order(causal):
+    # independent relative perturbations of size <= u of every numerator and denominator
+    # product, with u so large that u kappa_i reaches 0.9 on the worst row: every row moves by
+    # at most u cond_i / (1 - u kappa_i) of its max, the bound the parity metric uses
+    q, k, v = _qkv(48, 16, seed=53)
+    om = _orf(32, 16, seed=53)[0]
+    cond, kden = O.row_condition_head(q, k, v, om, O.TRIG, causal, with_den=True)
+    t = _terms(q, k, om, O.TRIG, causal)
+    base = O.favor_explicit_head(q, k, v, om, O.TRIG, causal)
+    u = 0.9 / kden.max()
+    rng = np.random.default_rng(5)
+    worst = 0.0
+    for trial in range(4):
+        # trial 0 pushes every product against its row's denominator; the rest are random
+        if trial == 0:
+            ed = -np.sign(t.sum(axis=(1, 2)))[:, None, None] * np.sign(t)
+        else:
+            ed = rng.uniform(-1, 1, t.shape)
+        en = rng.uniform(-1, 1, t.shape + (v.shape[1],))
+        num = np.einsum("ifj,ifjn,jn->in", t, 1 + u * en, v)
+        den = (t * (1 + u * ed)).sum(axis=(1, 2))
+        out = num / den[:, None]
+        bound = u * cond / (1 - u * kden)
+        ratio = np.abs(out - base).max(axis=1) / (np.abs(base).max(axis=1) * bound)
+        worst = max(worst, ratio.max())
+    assert worst <= 1.0 + 1e-9
+
+
+@pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
+@pytest.mark.parametrize("causal", [False, True])
+def test_rounding_terms_match_monte_carlo(kind, causal):
+    # perturb one level's operands by independent N(0, s^2) relative errors and recompute
+    # num and den by brute force: their sample variances over the trials must equal s^2 times
+    # the level's sums of squares (4000 trials: the ratio's spread is about 2%)
+    L, d, M = 24, 8, 8
+    q, k, v = _qkv(L, d, seed=54)
+    om = _orf(M, d, seed=54)[0]
+    t = O.row_rounding_terms_head(q, k, v, om, kind, causal)
+    fq, fk = O.phi(q, om, kind), O.phi(k, om, kind)
+    mask = np.tril(np.ones((L, L))) if causal else np.ones((L, L))
+    # per-row states S_i, z_i over the keys each row sees
+    S = np.einsum("ij,jf,jn->ifn", mask, fk, v)
+    z = np.einsum("ij,jf->if", mask, fk)
+    A = (fq @ fk.T) * mask
+    s, T = 1e-7, 4000
+    rng = np.random.default_rng(11)
+    acc = {key: [] for key in ("1", "2", "3")}
+    for _ in range(T):
+        e1 = rng.standard_normal(fk.shape) * s
+        fk_p = fk * (1 + e1)
+        A1 = (fq @ fk_p.T) * mask
+        e2 = rng.standard_normal((L, L)) * s
+        A2 = A * (1 + e2)
+        e3 = rng.standard_normal(S.shape[1:]) * s
+        e3z = rng.standard_normal(z.shape[1:]) * s
+        n3 = np.einsum("if,ifn->in", fq, S * (1 + e3)[None])
+        d3 = np.einsum("if,if->i", fq, z * (1 + e3z)[None])
+        acc["1"].append(np.concatenate([A1 @ v, A1.sum(axis=1)[:, None]], axis=1))
+        acc["2"].append(np.concatenate([A2 @ v, A2.sum(axis=1)[:, None]], axis=1))
+        acc["3"].append(np.concatenate([n3, d3[:, None]], axis=1))
+    for lev in ("1", "2", "3"):
+        var = np.var(np.stack(acc[lev]), axis=0) / s ** 2
+        want = np.concatenate([t["N" + lev], t["D" + lev][:, None]], axis=1)
+        live = want > 1e-12 * want.max()
+        np.testing.assert_allclose(var[live], want[live], rtol=0.12)
+        assert np.all(var[~live] <= 1e-6 * want.max())
+    # and the values themselves
+    base = O.favor_explicit_head(q, k, v, om, kind, causal)
+    np.testing.assert_allclose(t["out"], base, rtol=1e-9, atol=1e-12 * np.abs(base).max())
+    np.testing.assert_allclose(t["den"], A.sum(axis=1), rtol=1e-9)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_rounding_terms_follow_the_asked_rows(causal):
+    q, k, v = _qkv(97, 16, seed=55)
+    om = _orf(32, 16, seed=55)[0]
+    rows = np.array([96, 3, 40, 3, 0, 77])
+    full = O.row_rounding_terms_head(q, k, v, om, O.TRIG, causal)
+    part = O.row_rounding_terms_head(q, k, v, om, O.TRIG, causal, rows)
+    for key in full:
+        np.testing.assert_allclose(part[key], full[key][rows], rtol=1e-12, atol=0)

@@ -16,7 +16,7 @@ import torch
 
 import favor_inputs as fi
 from oracle import favor_oracle as O
-from parity_util import TOL_BF16, U_BF16, check_rows
+from parity_util import TOL_BF16, U_BF16, U_BIDIR16, U_CAUSAL16, RowCond, check_rows
 
 
 def _bf16(x):
@@ -29,6 +29,17 @@ def _head(L, d=64, M=256, seed=0):
     om = O.orf_matrices(G, R, M).astype(np.float32)
     q, k, v = (fi.as_f64(fi.round_to(x, "bf16"))[0, 0] for x in (q, k, v))
     return q, k, v, fi.as_f64(fi.round_to(om, "bf16"))[0]
+
+
+def _cond(q, k, v, om, kind, causal):
+    """The RowCond the GPU tests pass, for one head, with a leading head axis."""
+    c, kd = O.row_condition_head(q, k, v, om, kind, causal, with_den=True)
+    t = O.row_rounding_terms_head(q, k, v, om, kind, causal)
+    return RowCond(c[None], kd[None], {key: val[None] for key, val in t.items()})
+
+
+def _u(causal):
+    return U_CAUSAL16 if causal else U_BIDIR16
 
 
 def _quadratic(fq, fk, v, causal, strict=False):
@@ -45,7 +56,7 @@ def _planted(kind, causal):
     q, k, v, om = _head(L)
     fq, fk = O.phi(q, om, kind), O.phi(k, om, kind)
     ref = O.favor_causal_head(q, k, v, om, kind) if causal else O.favor_bidirectional_head(q, k, v, om, kind)
-    cond = O.row_condition_head(q, k, v, om, kind, causal)
+    cond = _cond(q, k, v, om, kind, causal)
     bad = []
     if causal:
         bad.append(("strict mask", _quadratic(fq, fk, v, True, strict=True)))
@@ -65,10 +76,10 @@ def _planted(kind, causal):
 def test_planted_kernel_mistakes_are_rejected(kind, causal):
     ref, cond, bad = _planted(kind, causal)
     trig = kind == O.TRIG
-    check_rows(_bf16(ref)[None], ref[None], cond[None], TOL_BF16, U_BF16, "exact, rounded", trig=trig)
+    check_rows(_bf16(ref)[None], ref[None], cond, TOL_BF16, _u(causal), "exact, rounded", trig=trig)
     for name, got in bad:
         with pytest.raises(AssertionError):
-            check_rows(got[None], ref[None], cond[None], TOL_BF16, U_BF16, name, trig=trig)
+            check_rows(got[None], ref[None], cond, TOL_BF16, _u(causal), name, trig=trig)
 
 
 @pytest.mark.parametrize("kind", [O.TRIG, O.RELU])
@@ -83,9 +94,9 @@ def test_dropped_tail_tile_is_rejected(kind):
     fk_drop[31 * 128:] = 0.0
     for causal in ((False, True) if kind == O.RELU else (False,)):
         ref = _quadratic(fq, fk, v, causal)
-        cond = O.row_condition_head(q, k, v, om, kind, causal)
+        cond = _cond(q, k, v, om, kind, causal)
         with pytest.raises(AssertionError):
-            check_rows(_bf16(_quadratic(fq, fk_drop, v, causal))[None], ref[None], cond[None], TOL_BF16, U_BF16,
+            check_rows(_bf16(_quadratic(fq, fk_drop, v, causal))[None], ref[None], cond, TOL_BF16, _u(causal),
                        "tail dropped", trig=kind == O.TRIG)
 
 
@@ -99,3 +110,29 @@ def test_nonfinite_condition_takes_the_plain_tolerance():
     got[0, 0, 0] = 1.0
     with pytest.raises(AssertionError):
         check_rows(got, ref, cond, TOL_BF16, U_BF16, "nan cond", trig=True)
+
+
+def test_undetermined_rows_are_exempt_but_counted():
+    # u kappa = 0.5 and 0.99 take u cond / (headroom (1 - u kappa)); u kappa >= 1 is exempt from
+    # the per-row bound (counted) but not from the finiteness and median checks
+    u, cond = U_BF16, 1000.0
+    kden = np.array([[0.5, 0.99, 1.0, 3.0] + [1.0] * 5]) / u
+    rc = RowCond(np.full(kden.shape, cond), kden)
+    ref = np.ones((1, 9, 4))
+    got = ref.copy()
+    got[0, 0] += u * cond / 2 / 0.5 * 0.99       # just inside row 0's allowance
+    got[0, 3] += 1e6                               # undetermined: exempt
+    st = check_rows(got, ref, rc, TOL_BF16, u, "exempt", trig=True)
+    assert st["rows_undetermined"] == 7
+    bad = got.copy()
+    bad[0, 0] = ref[0, 0] + u * cond / 2 / 0.5 * 1.01
+    with pytest.raises(AssertionError):
+        check_rows(bad, ref, rc, TOL_BF16, u, "row 0 over", trig=True)
+    bad = got.copy()
+    bad[0, 5:] += 1.0                               # most rows off: the median check fails
+    with pytest.raises(AssertionError):
+        check_rows(bad, ref, rc, TOL_BF16, u, "median", trig=True)
+    bad = got.copy()
+    bad[0, 4, 0] = np.nan
+    with pytest.raises(AssertionError):
+        check_rows(bad, ref, rc, TOL_BF16, u, "nan", trig=True)
