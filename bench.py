@@ -551,6 +551,8 @@ def main():
     torch.cuda.synchronize()
     for i in range(args.warmup):
         step_graphs[i % N_SETS].replay()
+    for g in var_graphs:          # a graph's first replay uploads it: keep that out of the timing
+        g.replay()
     torch.cuda.synchronize()
 
     clocks = ClockSampler(local)
@@ -584,7 +586,7 @@ def main():
         raise RuntimeError("device status not OK after the timed region")
     # per-kernel average launch duration: each variant's graph (one launch per input set, back to
     # back) replayed between CUDA events on the launching stream
-    reps = max(1, min(args.steps, 200) // N_SETS)
+    reps = max(10, min(args.steps, 200) // N_SETS)
     per_variant = {}
     for j, (name, _, _) in enumerate(variants):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

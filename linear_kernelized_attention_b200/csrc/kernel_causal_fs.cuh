@@ -387,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         // intra(c) = P16 V_c
         if (!(ok = mbar_wait(bar(ms->p16_full), c & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(bar(ms->v_full[c & 1]), (c >> 1) & 1, abort_flag))) break;
         tc_fence_after();
         const uint64_t bv = d_v0 + uint64_t(((c & 1) * kTileB) >> 4);
         if (leader) {
