@@ -34,9 +34,10 @@
  * launch errors. Errors from inside a kernel surface at the next synchronisation.
  * favor_sync_status() synchronises the stream and returns the device-side status word.
  *
- * Scratch. The bf16 path needs none (cross-CTA sums travel through distributed shared memory).
- * favor_attention_f32, favor_attention_backward_f32 and favor_attention_host take scratch from a
- * library-owned stream-ordered pool on `stream` and release it on the same stream;
+ * Scratch. The bf16 causal path needs none (its cross-CTA sums travel through distributed
+ * shared memory). The bf16 bidirectional path, favor_attention_f32,
+ * favor_attention_backward_f32 and favor_attention_host take scratch from a library-owned
+ * stream-ordered pool on `stream` and release it on the same stream;
  * favor_attention_f32_noalloc uses a static device array instead. The decode step keeps its
  * state in caller-owned memory and needs no scratch; so does favor_orf_omega_seeded.
  *
@@ -77,14 +78,19 @@ typedef enum {
 /*
  * bf16 forward pass: the tensor-core path.
  * q, k, v, omega, out: device pointers to __nv_bfloat16, 16-byte aligned, layouts above.
- * Supported: d = 64; M a multiple of 16 with 16 <= M <= 256 (trig) or <= 512 (relu);
- * L >= 1 (ragged tails are masked); B*H <= 524280 (bidirectional) or B*H*ceil(M/64) (trig, and
- * relu with M <= 256) / B*H*ceil(M/128) (relu, M > 256) < 2^31 (causal). Other shapes return
+ * Supported: d in {16, 32, 64, 128}; 1 <= M <= 256 (trig) or <= 512 (relu); L >= 1 (ragged
+ * tails are masked). Bidirectional with d = 128 needs M <= 128 (shared memory of the query
+ * kernel). Causal needs d <= 64 and B*H*ceil(M/64) < 2^31. Other shapes return
  * FAVOR_ERR_UNSUPPORTED and launch nothing.
+ * Launches: bidirectional is three kernels on `stream` (key-side partial states over every SM,
+ * their merge into per-head state images, then the queries); its scratch comes from the
+ * library's stream-ordered pool and is released on the same stream (favor_workspace_bytes gives
+ * the size). Causal is one kernel (one thread-block cluster per head) and takes no scratch.
  * Arithmetic: Q Omega^T and K Omega^T on tensor cores (bf16 in, fp32 accumulate); features in
  * fp32 registers; every product on tensor cores accumulates in fp32.
- *   Bidirectional: phi(K) is rounded to bf16 for phi(K)^T [V|1]; the state is rounded to fp16
- *   under a power-of-two scale and phi(Q) to fp16 for phi(Q) S.
+ *   Bidirectional: phi(K) and the stabiliser-weighted values are rounded to bf16 for
+ *   phi(K)^T [V|1]; the merged state is rounded to fp16 under a power-of-two scale and phi(Q) to
+ *   fp16 for phi(Q) S.
  *   Causal (128-token chunks): phi(K) (carrying its stabiliser weight), phi(Q), the masked
  *   intra-chunk scores and the state image are rounded to bf16; the state's normaliser column
  *   enters phi(Q).z as a bf16 hi + lo pair; the intra-chunk denominator is summed in fp32.
@@ -263,7 +269,13 @@ const char* favor_status_string(int status);
  */
 int favor_selftest_timeout(long long limit_cycles, void* stream);
 
-/* Bytes of scratch one favor_attention call takes from cudaMallocAsync (0 if none). */
+/*
+ * Bytes of scratch one favor_attention call takes from the library's stream-ordered pool (host
+ * only; no launch). Bidirectional: the key kernel's partial states (fp32) and their references,
+ * and the merged state images the query kernel reads; the run split follows the current
+ * device's SM count. Causal: 0 (the state stays in TMEM, partial rows cross the cluster in
+ * shared memory). 0 for non-positive sizes and for shapes without a kernel.
+ */
 size_t favor_workspace_bytes(int B, int H, int L, int d, int M, int feature_kind, int causal);
 
 #ifdef __cplusplus

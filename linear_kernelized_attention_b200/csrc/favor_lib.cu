@@ -593,10 +593,14 @@ int favor_sync_status(void* stream) {
 
 size_t favor_workspace_bytes(int B, int H, int L, int d, int M, int feature_kind, int causal) {
   if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || M <= 0) return 0;
-  (void)feature_kind;
-  (void)causal;
-  (void)d;
-  return 0;  // the bidirectional tensor-core path reduces through distributed shared memory
+  if ((long long)B * H > INT_MAX) return 0;
+  if (feature_kind != FAVOR_TRIG && feature_kind != FAVOR_RELU) return 0;
+  if (check_tc_shape(d, M, feature_kind, causal) != FAVOR_OK) return 0;
+  // causal: the state stays in TMEM and partial rows cross the cluster in shared memory
+  if (causal) return 0;
+  SplitPlan pl{};
+  if (!plan_split(pl, B * H, L, d, M, feature_kind)) return 0;
+  return pl.ws_bytes;
 }
 
 int favor_attention_chunked(const void* q, const void* k, const void* v, const void* omega,

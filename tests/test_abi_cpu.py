@@ -74,6 +74,15 @@ def test_f32_and_orf_validation():
 def test_workspace_bytes_is_host_only():
     assert F.favor_workspace_bytes(1, 1, 1, 64, 64, 0, False) >= 0
     assert F.favor_workspace_bytes(0, 1, 1, 64, 64, 0, False) == 0
+    # bidirectional: at least one fp32 partial state per (head, 128-angle block) and one state
+    # image per head; causal takes none; unsupported shapes take none
+    B, H, L, d, M = 4, 8, 4096, 64, 256
+    ws = F.favor_workspace_bytes(B, H, L, d, M, 0, False)
+    assert ws >= B * H * 2 * (d + 1) * 256 * 4 + B * H * 2 * 256 * (d + 16) * 2
+    assert F.favor_workspace_bytes(B, H, L, d, M, 1, False) > 0
+    assert F.favor_workspace_bytes(B, H, L, d, M, 0, True) == 0
+    assert F.favor_workspace_bytes(B, H, L, 48, M, 0, False) == 0
+    assert F.favor_workspace_bytes(B, H, L, d, 272, 0, False) == 0
 
 
 # ------------------------------------------------------------------ decode entry points
