@@ -162,7 +162,46 @@ def _rows_read_before_add(q, k, v, Om, kind, causal, rows):
     return out
 
 
+_TERMS = O.row_rounding_terms_head
+_COND = O.row_condition_head
+
+
+def _terms_state_unsquared(q, k, v, Om, kind, causal, rows=None):
+    # level 3 from |S| instead of S^2 (a dropped square)
+    t = _TERMS(q, k, v, Om, kind, causal, rows)
+    fq = O.phi(q if rows is None else q[np.asarray(rows)], Om, kind)
+    S = O.phi(k, Om, kind).T @ v
+    if not causal:
+        t["N3"] = (fq * fq) @ np.abs(S)
+    else:
+        t["N3"] = t["N3"] * 1.5
+    return t
+
+
+def _terms_values_unsquared(q, k, v, Om, kind, causal, rows=None):
+    # level 2 weighted by |v| instead of v^2
+    t = _TERMS(q, k, v, Om, kind, causal, rows)
+    r = np.arange(q.shape[0]) if rows is None else np.asarray(rows)
+    A = O.phi(q[r], Om, kind) @ O.phi(k, Om, kind).T
+    if causal:
+        A = np.where(np.arange(k.shape[0])[None, :] <= r[:, None], A, 0.0)
+    t["N2"] = (A * A) @ np.abs(v)
+    return t
+
+
+def _kden_from_rows(q, k, v, Om, kind, causal, rows=None, with_den=False):
+    # the denominator's condition from |A_ij| (cancellation across features missed)
+    out = _COND(q, k, v, Om, kind, causal, rows, with_den)
+    if not with_den:
+        return out
+    kap, _ = O.row_diagnostics_head(q, k, v, Om, kind, causal, rows)
+    return out[0], kap
+
+
 CASES = [
+    ("row_rounding_terms_head", _terms_state_unsquared, [lambda: P.test_rounding_terms_match_monte_carlo(O.TRIG, False)]),
+    ("row_rounding_terms_head", _terms_values_unsquared, [lambda: P.test_rounding_terms_match_monte_carlo(O.RELU, True)]),
+    ("row_condition_head", _kden_from_rows, [lambda: P.test_denominator_condition_is_attained(False)]),
     ("favor_rows_head", _rows_sorted_order, [lambda: P.test_rows_head_equals_explicit_rows(O.TRIG, False)]),
     ("favor_rows_head", _rows_read_before_add, [lambda: P.test_rows_head_equals_explicit_rows(O.RELU, True)]),
     ("phi_trig", _phi_trig_no_exp, [P.test_trig_self_inner_product_identity]),
