@@ -116,9 +116,9 @@ def test_undetermined_rows_are_exempt_but_counted():
     # u kappa = 0.5 and 0.99 take u cond / (headroom (1 - u kappa)); u kappa >= 1 is exempt from
     # the per-row bound (counted) but not from the finiteness and median checks
     u, cond = U_BF16, 1000.0
-    kden = np.array([[0.5, 0.99, 1.0, 3.0] + [1.0] * 5]) / u
+    kden = np.array([[0.5, 0.99, 1.0, 3.0] + [1.0] * 5 + [0.0] * 90]) / u
     rc = RowCond(np.full(kden.shape, cond), kden)
-    ref = np.ones((1, 9, 4))
+    ref = np.ones((1, 99, 4))
     got = ref.copy()
     got[0, 0] += u * cond / 2 / 0.5 * 0.99       # just inside row 0's allowance
     got[0, 3] += 1e6                               # undetermined: exempt
@@ -130,6 +130,14 @@ def test_undetermined_rows_are_exempt_but_counted():
         check_rows(bad, ref, rc, TOL_BF16, u, "row 0 over", trig=True)
     bad = got.copy()
     bad[0, 5:] += 1.0                               # most rows off: the median check fails
+    with pytest.raises(AssertionError):
+        check_rows(bad, ref, rc, TOL_BF16, u, "median", trig=True)
+    # more than the allowed share of exempt rows fails on its own
+    many = RowCond(rc.cond, np.where(np.arange(99) < 20, 2.0 / u, 0.0)[None])
+    with pytest.raises(AssertionError):
+        check_rows(got, ref, many, TOL_BF16, u, "share", trig=True)
+    bad = got.copy()
+    bad[0, 5:] += 1.0
     with pytest.raises(AssertionError):
         check_rows(bad, ref, rc, TOL_BF16, u, "median", trig=True)
     bad = got.copy()
