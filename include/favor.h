@@ -270,6 +270,16 @@ const char* favor_status_string(int status);
 int favor_selftest_timeout(long long limit_cycles, void* stream);
 
 /*
+ * Self-test of the FMA-pipe sine and cosine the trig kernels can use in place of the SFU's (no
+ * counterpart on the pages; the method is a Cody-Waite reduction by pi and minimax polynomials on
+ * [-pi/2, pi/2], coefficients derived in csrc/sincos_coeffs.py). u, sin_out, cos_out: device
+ * pointers to n floats, 4-byte aligned; sin_out[i] and cos_out[i] receive sin(u[i]) and cos(u[i]).
+ * Accurate to 1e-6 (sin) and 2e-7 (cos) absolute for |u| <= 400. Errors: FAVOR_ERR_NULL,
+ * FAVOR_ERR_SHAPE (n <= 0), FAVOR_ERR_ALIGN, FAVOR_ERR_DEVICE, FAVOR_ERR_CUDA.
+ */
+int favor_selftest_sincos(const float* u, float* sin_out, float* cos_out, int n, void* stream);
+
+/*
  * Bytes of scratch one favor_attention call takes from the library's stream-ordered pool (host
  * only; no launch). Bidirectional: the key kernel's partial states (fp32) and their references,
  * and the merged state images the query kernel reads; the run split follows the current

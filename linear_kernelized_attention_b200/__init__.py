@@ -7,7 +7,8 @@ if the library is missing or a call fails, an exception is raised.
 Entry points mirror the C ABI in include/favor.h:
     favor_attention, favor_attention_chunked, favor_attention_f32, favor_orf_omega,
     favor_attention_host, favor_sync_status, favor_status_string, favor_workspace_bytes,
-    favor_selftest_timeout, favor_attention_f32_noalloc, favor_noalloc_scratch_bytes,
+    favor_selftest_timeout, favor_selftest_sincos, favor_attention_f32_noalloc,
+    favor_noalloc_scratch_bytes,
     favor_decode_state_bytes, favor_decode_init, favor_decode_step, favor_orf_omega_seeded,
     favor_orf_gaussians_seeded, favor_philox4x64, favor_attention_backward_f32
 """
@@ -35,6 +36,7 @@ _SIGS = {
     "favor_sync_status": (_i, [_vp]),
     "favor_status_string": (ctypes.c_char_p, [_i]),
     "favor_selftest_timeout": (_i, [_ll, _vp]),
+    "favor_selftest_sincos": (_i, [_vp] * 3 + [_i, _vp]),
     "favor_workspace_bytes": (_sz, [_i] * 7),
     "favor_attention_f32_noalloc": (_i, [_vp] * 5 + [_i] * 7 + [_vp]),
     "favor_noalloc_scratch_bytes": (_sz, []),
@@ -216,6 +218,18 @@ def favor_workspace_bytes(B, H, L, d, M, feature_kind=FAVOR_TRIG, causal=False) 
 
 def favor_selftest_timeout(limit_cycles: int, stream=None) -> int:
     return lib().favor_selftest_timeout(int(limit_cycles), _stream(stream))
+
+
+def favor_selftest_sincos(u, stream=None):
+    """FMA-pipe (sin(u), cos(u)) of a contiguous float32 CUDA tensor, as two new tensors."""
+    import torch
+    if u.dtype != torch.float32 or not u.is_cuda or not u.is_contiguous():
+        raise ValueError("u must be a contiguous float32 CUDA tensor")
+    s, c = torch.empty_like(u), torch.empty_like(u)
+    rc = lib().favor_selftest_sincos(u.data_ptr(), s.data_ptr(), c.data_ptr(), u.numel(), _stream(stream))
+    if rc != 0:
+        raise FavorError(rc, "favor_selftest_sincos")
+    return s, c
 
 
 def favor_attention_f32_noalloc(q, k, v, omega, out=None, feature_kind=FAVOR_TRIG, causal=False,

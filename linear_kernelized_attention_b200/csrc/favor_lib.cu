@@ -33,6 +33,18 @@ __global__ void k_selftest_timeout(long long limit_cycles) {
   mbar_wait(smem_u32(&b), 0, nullptr, limit_cycles);
   __syncthreads();
 }
+
+// The FMA-pipe sine and cosine (sincos_poly.cuh) of n angles, one per thread, so that tests can
+// hold the device evaluation against the mathematics and the kernels' SFU alternative.
+__global__ void k_selftest_sincos(const float* __restrict__ u, float* __restrict__ s, float* __restrict__ c,
+                                  int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float sv, cv;
+  sincos_fma(u[i], sv, cv);
+  s[i] = sv;
+  c[i] = cv;
+}
 }  // namespace favor
 
 namespace {
@@ -814,6 +826,18 @@ int favor_selftest_timeout(long long limit_cycles, void* stream) {
   if (rc != FAVOR_OK) return rc;
   if (limit_cycles <= 0 || limit_cycles > 4000000000ll) return FAVOR_ERR_SHAPE;
   favor::k_selftest_timeout<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles);
+  return cudaGetLastError() == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
+}
+
+int favor_selftest_sincos(const float* u, float* sin_out, float* cos_out, int n, void* stream) {
+  if (!u || !sin_out || !cos_out) return FAVOR_ERR_NULL;
+  if (n <= 0) return FAVOR_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(u) | reinterpret_cast<uintptr_t>(sin_out) | reinterpret_cast<uintptr_t>(cos_out)) &
+      3u)
+    return FAVOR_ERR_ALIGN;
+  int rc = check_device();
+  if (rc != FAVOR_OK) return rc;
+  favor::k_selftest_sincos<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(u, sin_out, cos_out, n);
   return cudaGetLastError() == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
 

@@ -566,27 +566,57 @@ __global__ void __launch_bounds__(256) k_bidir_merge(const MergeParams p) {
   const int rb = blockIdx.y;
   const long long bh = pr / p.nab;
   const int ab = (int)(pr % p.nab);
+  const int ns = min(nslots(pr, p), kMergeMaxSlots);
+  uint8_t* img = p.img + bh * p.img_bytes;
+  const float* part = p.part + pr * p.smax * (long long)(DP + 1) * R;
+  const long long sstride = (long long)(DP + 1) * R;
+  // The partial states do not depend on the weights: every thread starts loading slots 0 and 1
+  // of its first work item before the first warp has turned the metadata into weights.
+  const int w0 = threadIdx.x;
+  const bool pre = w0 < 4 * NV && (w0 >> 2) <= DP;
+  float4 pa0 = make_float4(0.f, 0.f, 0.f, 0.f), pa1 = pa0, pb0 = pa0, pb1 = pa0;
+  if (pre) {
+    const float* src = part + (long long)(w0 >> 2) * R + rb * 32 + (w0 & 3) * 8;
+    if (ns > 0) {
+      pa0 = *reinterpret_cast<const float4*>(src);
+      pa1 = *reinterpret_cast<const float4*>(src + 4);
+    }
+    if (ns > 1) {
+      pb0 = *reinterpret_cast<const float4*>(src + sstride);
+      pb1 = *reinterpret_cast<const float4*>(src + sstride + 4);
+    }
+  }
   if (threadIdx.x < 32) {
-    // the head's reference (max over its slots) and the bound of its merged state
+    // the head's reference (max over its slots) and the bound of its merged state; a lane holds
+    // slots lane and lane + 32 of each of the head's (at most 4) angle blocks
     const int lane = threadIdx.x;
+    float mc[8], mb[8];
     float cmax = -INFINITY;
-    for (int a2 = 0; a2 < p.nab; ++a2) {
-      const long long q2 = bh * p.nab + a2;
-      const int ns = nslots(q2, p);
-      for (int s = lane; s < ns; s += 32) cmax = fmaxf(cmax, KIND == 0 ? p.meta[(q2 * p.smax + s) * 2] : 0.f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int a2 = e >> 1, sl = lane + 32 * (e & 1);
+      mc[e] = -INFINITY;
+      mb[e] = 0.f;
+      if (a2 < p.nab) {
+        const long long q2 = bh * p.nab + a2;
+        if (sl < nslots(q2, p)) {
+          const float* m = p.meta + (q2 * p.smax + sl) * 2;
+          mc[e] = KIND == 0 ? m[0] : 0.f;
+          mb[e] = m[1];
+        }
+      }
+      cmax = fmaxf(cmax, mc[e]);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
     float bound = 0.f;
-    for (int a2 = 0; a2 < p.nab; ++a2) {
-      const long long q2 = bh * p.nab + a2;
-      const int ns = nslots(q2, p);
-      for (int s = lane; s < ns; s += 32) {
-        const float* m = p.meta + (q2 * p.smax + s) * 2;
-        const float w = KIND == 0 ? __expf(m[0] - cmax) : 1.f;
-        bound += w * m[1];
-        if (a2 == ab && s < kMergeMaxSlots) wts[s] = w;
-      }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int a2 = e >> 1, sl = lane + 32 * (e & 1);
+      if (mc[e] == -INFINITY) continue;
+      const float w = KIND == 0 ? __expf(mc[e] - cmax) : 1.f;
+      bound += w * mb[e];
+      if (a2 == ab) wts[sl] = w;
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) bound += __shfl_xor_sync(0xffffffffu, bound, o);
@@ -594,10 +624,6 @@ __global__ void __launch_bounds__(256) k_bidir_merge(const MergeParams p) {
   }
   __syncthreads();
   const float scale = scale_s;
-  const int ns = min(nslots(pr, p), kMergeMaxSlots);
-  uint8_t* img = p.img + bh * p.img_bytes;
-  const float* part = p.part + pr * p.smax * (long long)(DP + 1) * R;
-  const long long sstride = (long long)(DP + 1) * R;
   // one work item = 8 consecutive state rows of one value row: two float4 loads per slot, and 8
   // consecutive features of the image, i.e. one 16-byte chunk
   for (int w = threadIdx.x; w < 4 * NV; w += blockDim.x) {
@@ -607,6 +633,19 @@ __global__ void __launch_bounds__(256) k_bidir_merge(const MergeParams p) {
     if (nn <= DP) {
       const float* src = part + (long long)nn * R + r0;
       int s = 0;
+      if (w == w0) {
+        // slots 0 and 1, loaded before the weights were known
+        const float wa = ns > 0 ? wts[0] : 0.f, wb = ns > 1 ? wts[1] : 0.f;
+        v[0] = fmaf(wa, pa0.x, wb * pb0.x);
+        v[1] = fmaf(wa, pa0.y, wb * pb0.y);
+        v[2] = fmaf(wa, pa0.z, wb * pb0.z);
+        v[3] = fmaf(wa, pa0.w, wb * pb0.w);
+        v[4] = fmaf(wa, pa1.x, wb * pb1.x);
+        v[5] = fmaf(wa, pa1.y, wb * pb1.y);
+        v[6] = fmaf(wa, pa1.z, wb * pb1.z);
+        v[7] = fmaf(wa, pa1.w, wb * pb1.w);
+        s = min(ns, 2);
+      }
       for (; s + 2 <= ns; s += 2) {
         const float4 a0 = *reinterpret_cast<const float4*>(src + s * sstride);
         const float4 a1 = *reinterpret_cast<const float4*>(src + s * sstride + 4);
