@@ -88,7 +88,7 @@ struct StateCfg {
   static constexpr int NV = DP + 16;                         // MMA2 N: values, normaliser (column DP), pad
   static constexpr int NSB = KIND == 0 ? 2 : 1;              // 128-row state blocks (trig: cos, sin)
   static constexpr int R = 128 * NSB;                        // state rows of a pair
-  static constexpr int NBUF = (KIND == 0 && DP == 128) ? 3 : 4;  // 64-key U/phi buffers
+  static constexpr int NBUF = (KIND == 0 && DP == 128) ? 3 : 5;  // 64-key U/phi buffers
   static constexpr int NS = DP == 64 ? 4 : 2;                // K/V stages
   static constexpr int kStageB = (2 * NCB + 1) * kBoxB;      // V boxes | column box | K boxes
   static constexpr int kOmB = NCB * kBoxB;                   // one Omega block
@@ -117,7 +117,7 @@ struct alignas(16) StateMisc {
   float redmax[2][8];
   uint64_t om_full[2], om_free[2];
   uint64_t kv_full[4], kv_empty[4], w_full[4];
-  uint64_t u_full[4], p_full[4], buf_free[4];
+  uint64_t u_full[5], p_full[5], buf_free[5];
   uint64_t s_done, s_free, drain;
   uint64_t norm_sync;  // bounded barrier among the 128 norm threads
 };
@@ -246,24 +246,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (whole warp; the
-    // elected lane issues the MMAs and commits)
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ projection issuer (whole warp;
+    // the elected lane issues): U^T = Omega_a K_item^T into buffer it % NBUF as soon as the state
+    // product of item it - NBUF has released that buffer, so the epilogue warps find the next
+    // item's angles ready instead of waiting for the state products in between
     if (n > 0) {
       const bool leader = elect_one();
       const uint32_t id1 = idesc_f16(128, 64, 1, 1, 0, 0);
-      const uint32_t id2 = idesc_f16(128, NV, 1, 1, 0, 1);
       const int nitems = 2 * n;
-      bool ok = true;
-      RunWalker w1(tt0, n, nt), w2(tt0, n, nt);  // the projection stream and the state stream
-      auto mma1 = [&](int it) -> bool {
+      RunWalker w1(tt0, n, nt);
+      for (int it = 0; it < nitems; ++it) {
         const int t = it >> 1, hf = it & 1, s = t % NS, b = it % NBUF;
         w1.advance_to(t);
         const int pk = w1.k;
         if (hf == 0) {
-          if (w1.first() && !mbar_wait(bar(ms->om_full[pk & 1]), (pk >> 1) & 1, abort_flag)) return false;
-          if (!mbar_wait(bar(ms->kv_full[s]), (t / NS) & 1, abort_flag)) return false;
+          if (w1.first() && !mbar_wait(bar(ms->om_full[pk & 1]), (pk >> 1) & 1, abort_flag)) break;
+          if (!mbar_wait(bar(ms->kv_full[s]), (t / NS) & 1, abort_flag)) break;
         }
+        if (it >= NBUF && !mbar_wait(bar(ms->buf_free[b]), ((it - NBUF) / NBUF) & 1, abort_flag)) break;
         tc_fence_after();
         const uint64_t a0 = sdesc_sw128(s_om + (pk & 1) * C::kOmB, 16, 1024);
         const uint64_t b0 = sdesc_sw128(s_stage + s * C::kStageB + (NCB + 1) * kBoxB + hf * 64 * kRowB, 16, 1024);
@@ -280,8 +281,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (hf == 1 && w1.last()) mma_commit(bar(ms->om_free[pk & 1]));
         }
         __syncwarp();
-        return true;
-      };
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ state-product issuer (whole
+    // warp; the elected lane issues the MMAs and commits)
+    if (n > 0) {
+      const bool leader = elect_one();
+      const uint32_t id2 = idesc_f16(128, NV, 1, 1, 0, 1);
+      const int nitems = 2 * n;
+      bool ok = true;
+      RunWalker w2(tt0, n, nt);
       auto write_meta_max = [&](int pk) {
         float mx = 0.f;
         for (int w = 0; w < 8; ++w) mx = fmaxf(mx, ms->redmax[pk & 1][w]);
@@ -291,10 +302,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (KIND == 1) p.meta[sl * 2] = 0.f;
         }
       };
-      // projections run NBUF - 1 items ahead: the projection issued after item it's state product
-      // goes to the buffer item it - 1 used, whose product has long completed, so the tensor pipe
-      // gets both back to back and never drains waiting on the product just issued
-      for (int it = 0; ok && it < NBUF - 1 && it < nitems; ++it) ok = mma1(it);
       for (int it = 0; ok && it < nitems; ++it) {
         const int t = it >> 1, hf = it & 1, s = t % NS, b = it % NBUF;
         w2.advance_to(t);
@@ -326,12 +333,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         __syncwarp();
-        const int nx = it + NBUF - 1;
-        if (nx < nitems) {
-          if (it >= 1 && !(ok = mbar_wait(bar(ms->buf_free[(it - 1) % NBUF]), ((it - 1) / NBUF) & 1, abort_flag)))
-            break;
-          if (!(ok = mma1(nx))) break;
-        }
       }
       if (ok) {
         w2.advance_to(n - 1);
@@ -821,27 +822,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (whole warp; the
-    // elected lane issues the MMAs and commits)
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ projection issuer (whole warp;
+    // the elected lane issues): U = Q_tile Omega_ab^T into buffer j % NBQ once the state product
+    // of item j - NBQ has released it; a new head's first projection waits for its Omega
     if (n > 0) {
       const bool leader = elect_one();
       const uint32_t id1 = idesc_f16(128, 128, 1, 1, 0, 0);
-      const uint32_t fmt = KIND == 0 ? 0u : 1u;  // fp16 (trig) or bf16 (ReLU) state operands
-      const uint32_t id2 = idesc_f16(128, NV, fmt, fmt, 0, 0);
       const int nit = n * nab;
       const uint64_t om0 = sdesc_sw128(s_om, 16, 1024);
-      const uint64_t img0 = sdesc_sw128(s_img, 16, 1024);
-      bool ok = true;
-      RunWalker w1(tt0, n, nt), w2(tt0, n, nt), w3(tt0, n, nt);  // projections, state products, look-ahead
-      auto mma1 = [&](int j) -> bool {
+      RunWalker w1(tt0, n, nt);
+      for (int j = 0; j < nit; ++j) {
         const int t = j / nab, ab = j - t * nab, b = j % NBQ, s = t & 1;
         w1.advance_to(t);
         if (ab == 0) {
-          if (!mbar_wait(bar(ms->q_full[s]), (t >> 1) & 1, abort_flag)) return false;
-          if (w1.first() && !mbar_wait(bar(ms->head_full), w1.k & 1, abort_flag)) return false;
+          if (!mbar_wait(bar(ms->q_full[s]), (t >> 1) & 1, abort_flag)) break;
+          if (w1.first() && !mbar_wait(bar(ms->head_full), w1.k & 1, abort_flag)) break;
         }
-        if (j >= NBQ && !mbar_wait(bar(ms->buf_free[b]), ((j - NBQ) / NBQ) & 1, abort_flag)) return false;
+        if (j >= NBQ && !mbar_wait(bar(ms->buf_free[b]), ((j - NBQ) / NBQ) & 1, abort_flag)) break;
         tc_fence_after();
         const uint64_t q0 = sdesc_sw128(s_q + s * NCB * kBoxB, 16, 1024);
         if (leader) {
@@ -855,15 +853,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ab == nab - 1) mma_commit(bar(ms->q_empty[s]));
         }
         __syncwarp();
-        return true;
-      };
-      int nx = 0;  // next item whose projection is to be issued
-      // projections run NBQ - 1 items ahead, into buffers whose products completed an item earlier
-      while (ok && nx < nit && nx < NBQ - 1) {
-        w3.advance_to(nx / nab);
-        if (w3.k != 0) break;
-        ok = mma1(nx++);
       }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ state-product issuer (whole
+    // warp; the elected lane issues the MMAs and commits)
+    if (n > 0) {
+      const bool leader = elect_one();
+      const uint32_t fmt = KIND == 0 ? 0u : 1u;  // fp16 (trig) or bf16 (ReLU) state operands
+      const uint32_t id2 = idesc_f16(128, NV, fmt, fmt, 0, 0);
+      const int nit = n * nab;
+      const uint64_t img0 = sdesc_sw128(s_img, 16, 1024);
+      bool ok = true;
+      RunWalker w2(tt0, n, nt);
       for (int j = 0; ok && j < nit; ++j) {
         const int t = j / nab, ab = j - t * nab, b = j % NBQ, nb = t % NBN;
         w2.advance_to(t);
@@ -885,14 +888,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (head_end) mma_commit(bar(ms->head_free));
         }
         __syncwarp();
-        // projections ahead: two items in flight, and none past a head change until the head's
-        // last state product has been issued (the next head's Omega and image replace these)
-        while (ok && nx < nit && nx <= j + NBQ - 1) {
-          w3.advance_to(nx / nab);
-          const int hn = w3.k, hc = w2.k;
-          if (!(hn == hc || (head_end && hn == hc + 1))) break;
-          ok = mma1(nx++);
-        }
       }
       if (leader) mma_commit(bar(ms->drain));
       __syncwarp();
