@@ -49,9 +49,11 @@ constexpr float kMargin = 16.f;     // stabiliser head-room above the largest |k
 constexpr int kThreads = 512;
 
 // Angles of 8 consecutive ones evaluated on the FMA pipe (bit j set: angle j of the group);
-// the rest go to the SFU. 0x00 (all on the SFU) measured fastest here: the kernels are bound by MMA issue and latency, not the SFU.
+// the rest go to the SFU. With the projections issued by their own warp the feature warps are
+// busy enough for the SFU to matter: 0x11 (two angles in eight on the FMA pipe) measured fastest,
+// ahead of 0x00, 0x01, 0x15, 0x41 and 0x55.
 #ifndef FAVOR_POLY_MASK
-#define FAVOR_POLY_MASK 0x00u
+#define FAVOR_POLY_MASK 0x11u
 #endif
 constexpr uint32_t kPolyMask = FAVOR_POLY_MASK;
 
