@@ -42,11 +42,11 @@
 //              phi(Q).z with z split into bf16 hi and lo rows, intra = P16 V_c
 // The intra denominator sum_j P16_ij is accumulated in fp32 registers.
 //
-// Warp roles (544 threads): 0 TMA; 1 TMEM allocator and issuer A (U_K(c + 1) is issued before
+// Warp roles (640 threads): 0 TMA; 1 TMEM allocator and issuer A (U_K(c + 1) is issued before
 // the state update of chunk c); 2 issuer B; 3 key norms and references; 4-7 phi'(K) (thread =
 // key row); 8-11 the state image, then phi(Q) (thread = feature row, then query row; two phi(Q)
 // slots, so the next chunk's features overlap this chunk's products); 12-15 P16 and partial rows
-// (thread = query row); 16 combiner of the owned rows.
+// (thread = query row); 16-19 combiner of the owned rows (thread = a quarter of a row).
 // Head sizes 16 and 32 ride in the 64-column boxes (zeros past d).
 #pragma once
 #include <cuda_bf16.h>
@@ -60,7 +60,7 @@ namespace cf {
 constexpr int kTile = 128;
 constexpr int kRowB = 128;
 constexpr int kTileB = kTile * kRowB;  // 16 KB
-constexpr int kThreads = 544;
+constexpr int kThreads = 640;
 #ifndef FAVOR_POLY_MASK_CAUSAL
 #define FAVOR_POLY_MASK_CAUSAL 0x00u
 #endif
@@ -116,6 +116,7 @@ struct alignas(16) CausalMisc {
   uint64_t img_full, img_free, s_ready, p16_full, pr_free;
   uint64_t phik_full[2], phik_free[2];  // per phi(K) buffer
   uint64_t recv_full[2], recv_free[2];  // per deposit buffer
+  uint64_t comb_sync;                   // bounded barrier among the 128 combiner threads
 };
 static_assert(sizeof(CausalMisc) <= 1024, "causal misc block");
 
@@ -196,6 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(ms->s_ready), 4);
     mbar_init(bar(ms->p16_full), 4);
     mbar_init(bar(ms->pr_free), 4);
+    mbar_init(bar(ms->comb_sync), 128);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -781,44 +783,67 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (G > 1 && pend >= 0) mbar_arrive_remote(mapa_shared(smem_u32(&ms->recv_full[pend & 1]), owner));
   } else if (G > 1) {
-    // ------------------------------------------------------------ combiner (warp 16)
+    // ------------------------------------------------------------ combiner (warps 16-19)
     // The owned rows of every chunk (16-row blocks b with b % G == g): the G partial rows,
     // summed in CTA order, divided and stored; every depositor may reuse its buffer once all
-    // owners have read it.
-    const int nown = kTile / G;  // owned rows per chunk
+    // owners have read it. Thread t takes 16 of the 64 columns of owned row t / 4 (G = 2 owns 64
+    // rows and takes them in two passes; G = 8 owns 16). The buffer is released as soon as every
+    // owned row is in registers, before the output stores.
+    const int t = tid - 16 * 32;
+    const int qq = t & 3, nown = kTile / G;
+    const bool cols = 16 * qq < p.d;
+    uint32_t cph = 0;  // phase of comb_sync
     bool ok = true;
     for (int c = 0; ok && c < nch; ++c) {
       const int pb = c & 1;
       if (!(ok = mbar_wait_cluster(bar(ms->recv_full[pb]), (c >> 1) & 1, abort_flag))) break;
-      // owned row ro (< 64 for G >= 2): 16-row block bi of the owned ones, row rr of it
-#pragma unroll 1
-      for (int ro = lane; ro < nown; ro += 32) {
-        const int bi = ro >> 4, rr = ro & 15;
-        float acc[64], den = 0.f;
+      float acc[2][16], den[2] = {0.f, 0.f};
 #pragma unroll
-        for (int e = 0; e < 64; ++e) acc[e] = 0.f;
-        for (int s = 0; s < G; ++s) {
-          const uint8_t* src = gb + kC_RECV + pb * kRecvBufB + ((bi * G + s) * 16 + rr) * kRecvRowB;
+      for (int ps = 0; ps < 2; ++ps) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint4 x = *reinterpret_cast<const uint4*>(src + 16 * e);
-            const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+        for (int e = 0; e < 16; ++e) acc[ps][e] = 0.f;
+        const int ro = 32 * ps + (t >> 2);
+        if (ro < nown && cols) {
+          const int bi = ro >> 4, rr = ro & 15;
+          for (int s = 0; s < G; ++s) {
+            const uint8_t* src = gb + kC_RECV + pb * kRecvBufB + ((bi * G + s) * 16 + rr) * kRecvRowB;
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              acc[8 * e + 2 * t] += __uint_as_float(w4[t] << 16);
-              acc[8 * e + 2 * t + 1] += __uint_as_float(w4[t] & 0xFFFF0000u);
+            for (int e = 0; e < 2; ++e) {
+              const uint4 x = *reinterpret_cast<const uint4*>(src + 32 * qq + 16 * e);
+              const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                acc[ps][8 * e + 2 * u] += __uint_as_float(w4[u] << 16);
+                acc[ps][8 * e + 2 * u + 1] += __uint_as_float(w4[u] & 0xFFFF0000u);
+              }
             }
+            den[ps] += *reinterpret_cast<const float*>(src + 128);
           }
-          den += *reinterpret_cast<const float*>(src + 128);
         }
-        const int token = c * kTile + (bi * G + g) * 16 + rr;
-        if (token < L) store_row(out + ((size_t)bh * L + token) * p.d, acc, den != 0.f ? 1.f / den : 0.f, p.d);
       }
-      // every owned row is read: release the buffer in every depositor (one fence, then relaxed
-      // arrives that do not wait for one another)
-      __syncwarp();
-      fence_acq_rel_cluster();
-      if (lane < G) mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&ms->recv_free[pb]), lane));
+      // every owned row is read: release the buffer in every depositor (one fence per releasing
+      // thread, then relaxed arrives that do not wait for one another)
+      if (!(ok = group_sync(bar(ms->comb_sync), cph, abort_flag))) break;
+      if (t < G) {
+        fence_acq_rel_cluster();
+        mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&ms->recv_free[pb]), t));
+      }
+#pragma unroll
+      for (int ps = 0; ps < 2; ++ps) {
+        const int ro = 32 * ps + (t >> 2);
+        if (ro >= nown || !cols) continue;
+        const int bi = ro >> 4, rr = ro & 15;
+        const int token = c * kTile + (bi * G + g) * 16 + rr;
+        if (token >= L) continue;
+        const float inv = den[ps] != 0.f ? 1.f / den[ps] : 0.f;
+        uint4* o = reinterpret_cast<uint4*>(out + ((size_t)bh * L + token) * p.d + 16 * qq);
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          o[e] = make_uint4(pack_bf16x2(acc[ps][8 * e] * inv, acc[ps][8 * e + 1] * inv),
+                            pack_bf16x2(acc[ps][8 * e + 2] * inv, acc[ps][8 * e + 3] * inv),
+                            pack_bf16x2(acc[ps][8 * e + 4] * inv, acc[ps][8 * e + 5] * inv),
+                            pack_bf16x2(acc[ps][8 * e + 6] * inv, acc[ps][8 * e + 7] * inv));
+      }
     }
   }
 
