@@ -510,8 +510,8 @@ int decode_cluster(long long BH, int M) {
 }
 
 // ------------------------------------------------------------------ ORF
-// One CTA per (d x d block, head): Gram-Schmidt in fp64 shared memory, rows scaled by chi
-// lengths. The Gaussians come from G and R, or (seeded) from the Philox stream of `seed`.
+// One CTA per (d x d block, head): panel-blocked Gram-Schmidt in fp64 shared memory, rows scaled
+// by chi lengths. The Gaussians come from G and R, or (seeded) from the Philox stream of `seed`.
 int launch_orf(const double* G, const double* R, void* omega, int H, int M, int d, int omega_dtype, uint64_t seed,
                int seeded, cudaStream_t st) {
   if (H <= 0 || M <= 0 || d <= 0) return FAVOR_ERR_SHAPE;
@@ -520,9 +520,9 @@ int launch_orf(const double* G, const double* R, void* omega, int H, int M, int 
   int rc = check_device();
   if (rc != FAVOR_OK) return rc;
   const int nb = (M + d - 1) / d;
-  const size_t smem = (size_t)d * d * sizeof(double);
+  const size_t smem = orf_smem_bytes(d);
   if ((rc = ensure_smem_attr(reinterpret_cast<const void*>(k_orf), (int)smem)) != FAVOR_OK) return rc;
-  k_orf<<<dim3(nb, H), 256, smem, st>>>(G, R, omega, H, M, d, omega_dtype, seed, seeded);
+  k_orf<<<dim3(nb, H), kOrfThreads, smem, st>>>(G, R, omega, H, M, d, omega_dtype, seed, seeded);
   return cudaGetLastError() == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
 

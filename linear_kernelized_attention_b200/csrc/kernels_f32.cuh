@@ -255,103 +255,210 @@ __global__ void __launch_bounds__(kThreads)
 }  // namespace f32
 
 // ------------------------------------------------------------------ ORF builder
-// One block per (head, d x d Gaussian block). Rows are orthonormalised in order by classical
-// Gram-Schmidt applied twice (fp64), then row r is scaled by |gauss_norms[h, r, :]|. With
-// `seeded`, the block's Gaussians and its rows' chi draws are generated here from `seed`
-// (philox.cuh: the same draws k_orf_gaussians writes out) instead of being read from G and R.
+// One block per (head, d x d Gaussian block). The block's rows are orthonormalised in order:
+// the Q factor of G^T = Q R with a positive diagonal R, which is what Gram-Schmidt in order
+// produces. Row r is then scaled by |gauss_norms[h, r, :]|. With `seeded`, the block's Gaussians
+// and its rows' chi draws are generated here from `seed` (philox.cuh: the same draws
+// k_orf_gaussians writes out) instead of being read from G and R.
 // "Masked Language Modeling for Proteins via Linearly Scalable Long-Context Transformers"
 // (方法详解) calls these orthogonal random features. The explainer's 核心机制 section
 // constrains the directions to a random subsample of an orthogonal matrix.
-__global__ void __launch_bounds__(256)
+//
+// Rows go in panels of kOrfPanel. A panel is first made orthogonal to every finished row by two
+// passes of block classical Gram-Schmidt (one warp per panel row, no block barrier), then
+// orthonormalised within itself by two passes of Cholesky QR on its Gram matrix (the lower
+// Cholesky factor L of V V^T gives V <- L^-1 V). Both are exact reformulations of Gram-Schmidt in
+// order (the same Q), in fp64; the serial chain is a few dozen small steps per panel instead of a
+// block-wide reduction per row.
+constexpr int kOrfThreads = 512;
+constexpr int kOrfPanel = 8;  // rows per panel: one warp each
+
+__host__ __device__ constexpr int orf_ld(int d) { return d | 1; }  // odd stride: conflict-free column reads
+__host__ __device__ constexpr size_t orf_smem_bytes(int d) {
+  return ((size_t)d * orf_ld(d) + kOrfPanel * 128 + kOrfPanel * kOrfPanel + kOrfPanel + 128) * sizeof(double);
+}
+
+__global__ void __launch_bounds__(kOrfThreads)
     k_orf(const double* __restrict__ G, const double* __restrict__ R, void* __restrict__ omega,
           int H, int M, int d, int out_bf16, uint64_t seed, int seeded) {
-  extern __shared__ double sq[];  // [d][d] rows being orthonormalised
-  __shared__ double dots[128];
-  __shared__ double snorm;
+  extern __shared__ double orf_sm[];
+  const int ld = orf_ld(d);
+  double* sq = orf_sm;                            // [d][ld] rows being orthonormalised
+  double* coef = sq + (size_t)d * ld;             // [kOrfPanel][128] coefficients against finished rows
+  double* gram = coef + kOrfPanel * 128;          // [kOrfPanel][kOrfPanel] Gram matrix -> Cholesky factor
+  double* rdiag = gram + kOrfPanel * kOrfPanel;   // [kOrfPanel] 1 / L_kk
+  double* chi = rdiag + kOrfPanel;                // [128] row lengths
   const int h = blockIdx.y, blk = blockIdx.x, nb = gridDim.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long n0 = (((long long)h * nb + blk) * d) * d;  // first draw of this block
   const long long NG = ((long long)H * nb * d * d + 3) / 4 * 4;
   if (seeded) {
-    for (long long gq = n0 / 4 + threadIdx.x; gq <= (n0 + d * d - 1) / 4; gq += blockDim.x) {
+    for (long long gq = n0 / 4 + tid; gq <= (n0 + d * d - 1) / 4; gq += blockDim.x) {
       double z[4];
       rng::normals4(seed, (uint64_t)gq, z);
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         const long long e = 4 * gq + p - n0;
-        if (e >= 0 && e < (long long)d * d) sq[e] = z[p];
+        if (e >= 0 && e < (long long)d * d) sq[(e / d) * ld + e % d] = z[p];
       }
     }
   } else {
     const double* g = G + n0;
-    for (int i = threadIdx.x; i < d * d; i += blockDim.x) sq[i] = g[i];
+    for (int e = tid; e < d * d; e += blockDim.x) sq[(e / d) * ld + e % d] = g[e];
+  }
+  // chi lengths: tpr threads per output row (a power of two <= 32), each summing every tpr-th
+  // group of four draws of the row
+  {
+    int lg = 0;
+    while ((1 << (lg + 1)) <= 32 && (d << (lg + 1)) <= (int)blockDim.x) ++lg;
+    const int tpr = 1 << lg, i = tid >> lg, part = tid & (tpr - 1);
+    const int r = blk * d + i;
+    double s = 0.0;
+    if (i < d && r < M) {
+      if (seeded) {
+        const long long nr = NG + ((long long)h * M + r) * d;
+        const long long g0 = nr / 4, g1 = (nr + d - 1) / 4;
+        for (long long gq = g0 + part; gq <= g1; gq += tpr) {
+          double z[4];
+          rng::normals4(seed, (uint64_t)gq, z);
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const long long n = 4 * gq + p;
+            if (n >= nr && n < nr + d) s = fma(z[p], z[p], s);
+          }
+        }
+      } else {
+        const double* rr = R + ((size_t)h * M + r) * d;
+        for (int t = part; t < d; t += tpr) s = fma(rr[t], rr[t], s);
+      }
+    }
+    for (int o = 1; o < tpr; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (part == 0 && i < d) chi[i] = sqrt(s);
   }
   __syncthreads();
-  // Row i: two classical Gram-Schmidt passes against rows 0 .. i-1, then normalisation.
-  // Dot products: 8 lanes per row j (32 rows per sweep). Update of v: kTpt lanes per column t,
-  // each summing every kTpt-th j, combined by shuffles (kTpt a power of two <= 32 dividing 32).
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int tpt = 1;
-  while (tpt * 2 <= 32 && tpt * 2 * d <= (int)blockDim.x) tpt *= 2;
-  const int sub8 = threadIdx.x & 7, grp = threadIdx.x >> 3, ngrp = blockDim.x >> 3;
-  const int col = threadIdx.x / tpt, part = threadIdx.x % tpt;
-  for (int i = 0; i < d; ++i) {
-    double* vi = sq + (size_t)i * d;
-    for (int pass = 0; pass < 2 && i > 0; ++pass) {
-      for (int j0 = 0; j0 < i; j0 += ngrp) {  // uniform trip count across the block
-        const int j = j0 + grp;
-        double s = 0.0;
-        if (j < i)
-          for (int t = sub8; t < d; t += 8) s = fma(sq[(size_t)j * d + t], vi[t], s);
-        s += __shfl_xor_sync(0xffffffffu, s, 4);
-        s += __shfl_xor_sync(0xffffffffu, s, 2);
-        s += __shfl_xor_sync(0xffffffffu, s, 1);
-        if (sub8 == 0 && j < i) dots[j] = s;
+
+  for (int r0 = 0; r0 < d; r0 += kOrfPanel) {
+    const int nr = min(kOrfPanel, d - r0);
+    const bool act = warp < nr;
+    double* vi = sq + (size_t)(r0 + warp) * ld;
+    // (1) two passes of classical Gram-Schmidt of panel row r0 + warp against rows 0 .. r0-1:
+    // lane l forms the coefficients of rows l, l+32, l+64, l+96, then owns columns l + 32 e
+    if (act && r0 > 0) {
+      const int nm = (r0 + 31) >> 5;  // warp-uniform
+      double* cw = coef + warp * 128;
+      for (int pass = 0; pass < 2; ++pass) {
+        double c[4] = {0.0, 0.0, 0.0, 0.0}, c2[4] = {0.0, 0.0, 0.0, 0.0};
+        const double* qr[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) qr[m] = sq + (size_t)min(lane + 32 * m, r0 - 1) * ld;
+        int t = 0;
+        for (; t + 1 < d; t += 2) {
+          const double x = vi[t], y = vi[t + 1];
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            if (m < nm) {
+              c[m] = fma(qr[m][t], x, c[m]);
+              c2[m] = fma(qr[m][t + 1], y, c2[m]);
+            }
+        }
+        if (t < d) {
+          const double x = vi[t];
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            if (m < nm) c[m] = fma(qr[m][t], x, c[m]);
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          if (lane + 32 * m < r0) cw[lane + 32 * m] = c[m] + c2[m];
+        __syncwarp();
+        double a[4] = {0.0, 0.0, 0.0, 0.0}, a2[4] = {0.0, 0.0, 0.0, 0.0};
+        for (int j = 0; j < r0; j += 2) {  // r0 is a multiple of the panel height, so even
+          const double cj = cw[j], ck = cw[j + 1];
+          const double* qj = sq + (size_t)j * ld;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (lane + 32 * e < d) {
+              a[e] = fma(cj, qj[lane + 32 * e], a[e]);
+              a2[e] = fma(ck, qj[ld + lane + 32 * e], a2[e]);
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (lane + 32 * e < d) vi[lane + 32 * e] -= a[e] + a2[e];
+        __syncwarp();
       }
-      __syncthreads();
-      double s = 0.0;
-      if (col < d)
-        for (int j = part; j < i; j += tpt) s = fma(dots[j], sq[(size_t)j * d + col], s);
-      for (int o = tpt >> 1; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (col < d && part == 0) vi[col] -= s;
-      __syncthreads();
-    }
-    if (warp == 0) {
-      double s = 0.0;
-      for (int t = lane; t < d; t += 32) s = fma(vi[t], vi[t], s);
-#pragma unroll
-      for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (lane == 0) snorm = sqrt(s);
     }
     __syncthreads();
-    for (int t = threadIdx.x; t < d; t += blockDim.x) vi[t] /= snorm;
-    __syncthreads();
-  }
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    const int r = blk * d + i;
-    if (r >= M) continue;
-    double s = 0.0;
-    if (seeded) {
-      const long long nr = NG + ((long long)h * M + r) * d;
-      for (long long gq = nr / 4; gq <= (nr + d - 1) / 4; ++gq) {
-        double z[4];
-        rng::normals4(seed, (uint64_t)gq, z);
+    // (2) two passes of Cholesky QR within the panel
+    for (int pass = 0; pass < 2; ++pass) {
+      if (act) {  // Gram row warp: <v_warp, v_k> for k <= warp
+        double g[kOrfPanel];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const long long n = 4 * gq + p;
-          if (n >= nr && n < nr + d) s = fma(z[p], z[p], s);
+        for (int k = 0; k < kOrfPanel; ++k) g[k] = 0.0;
+        for (int t = lane; t < d; t += 32) {
+          const double x = vi[t];
+#pragma unroll
+          for (int k = 0; k < kOrfPanel; ++k)
+            if (k <= warp) g[k] = fma(x, sq[(size_t)(r0 + k) * ld + t], g[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < kOrfPanel; ++k) {
+#pragma unroll
+          for (int o = 16; o; o >>= 1) g[k] += __shfl_xor_sync(0xffffffffu, g[k], o);
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int k = 0; k < kOrfPanel; ++k)
+            if (k <= warp) gram[warp * kOrfPanel + k] = g[k];
         }
       }
-    } else {
-      const double* rr = R + ((size_t)h * M + r) * d;
-      for (int t = 0; t < d; ++t) s = fma(rr[t], rr[t], s);
+      __syncthreads();
+      if (tid == 0) {  // lower Cholesky factor, in registers; rows past nr are the identity
+        double L[kOrfPanel][kOrfPanel];
+#pragma unroll
+        for (int a = 0; a < kOrfPanel; ++a)
+#pragma unroll
+          for (int b = 0; b <= a; ++b) L[a][b] = (a < nr) ? gram[a * kOrfPanel + b] : (a == b ? 1.0 : 0.0);
+        // right-looking: column c is scaled by 1/sqrt(pivot), then the trailing block loses its
+        // outer product, so the next pivot is ready after one update
+#pragma unroll
+        for (int c = 0; c < kOrfPanel; ++c) {
+          const double il = rsqrt(L[c][c]);
+          rdiag[c] = il;
+#pragma unroll
+          for (int a = c + 1; a < kOrfPanel; ++a) L[a][c] *= il;
+#pragma unroll
+          for (int a = c + 1; a < kOrfPanel; ++a)
+#pragma unroll
+            for (int b = c + 1; b <= a; ++b) L[a][b] = fma(-L[a][c], L[b][c], L[a][b]);
+        }
+#pragma unroll
+        for (int a = 0; a < kOrfPanel; ++a)
+#pragma unroll
+          for (int b = 0; b < a; ++b) gram[a * kOrfPanel + b] = L[a][b];
+      }
+      __syncthreads();
+      // V <- L^-1 V by forward substitution, one thread per column
+      for (int t = tid; t < d; t += blockDim.x) {
+        double q[kOrfPanel];
+#pragma unroll
+        for (int k = 0; k < kOrfPanel; ++k) {
+          if (k < nr) {
+            double x = sq[(size_t)(r0 + k) * ld + t];
+#pragma unroll
+            for (int j = 0; j < k; ++j) x = fma(-gram[k * kOrfPanel + j], q[j], x);
+            q[k] = x * rdiag[k];
+            sq[(size_t)(r0 + k) * ld + t] = q[k];
+          }
+        }
+      }
+      __syncthreads();
     }
-    dots[i] = sqrt(s);
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < d * d; e += blockDim.x) {
+  for (int e = tid; e < d * d; e += blockDim.x) {
     const int i = e / d, t = e % d, r = blk * d + i;
     if (r >= M) continue;
-    const double val = sq[e] * dots[i];
+    const double val = sq[(size_t)i * ld + t] * chi[i];
     const size_t o = ((size_t)h * M + r) * d + t;
     if (out_bf16)
       reinterpret_cast<__nv_bfloat16*>(omega)[o] = __double2bfloat16(val);
