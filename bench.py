@@ -41,17 +41,20 @@ METRIC = "FAVOR fwd tokens/s (B·H·L/s) at L=4096,d=64,M=256; % of tensor/HBM r
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of each variant's kernel
 # at this workload, from one ncu capture (profiles/), with the SHA-1 of the kernel sources the
 # capture was taken with. A value whose sources have changed since is reported as null.
-TRAFFIC = {"trig_causal": (51497216, "2faef9ca88a8fd89a38f55e1ff0c5241fbb7ed99")}
-KERNEL_SOURCES = ["linear_kernelized_attention_b200/csrc/ptx.cuh",
-                  "linear_kernelized_attention_b200/csrc/sincos_poly.cuh",
-                  "linear_kernelized_attention_b200/csrc/kernel_bidir_split.cuh",
-                  "linear_kernelized_attention_b200/csrc/kernel_causal_fs.cuh"]
+TRAFFIC = {"trig_causal": (51497216, "ff014ab33611f8622d9d069095ec8d10a98cec92")}
+_CSRC = "linear_kernelized_attention_b200/csrc/"
+_CAUSAL_SOURCES = [_CSRC + "ptx.cuh", _CSRC + "sincos_poly.cuh", _CSRC + "kernel_causal_fs.cuh"]
+_BIDIR_SOURCES = [_CSRC + "ptx.cuh", _CSRC + "sincos_poly.cuh", _CSRC + "kernel_bidir_split.cuh"]
+KERNEL_SOURCES = {"trig_causal": _CAUSAL_SOURCES, "relu_causal": _CAUSAL_SOURCES,
+                  "trig_bidir": _BIDIR_SOURCES, "relu_bidir": _BIDIR_SOURCES}
 
 
-def kernel_sources_sha():
+def kernel_sources_sha(variant):
+    """sha1 of the sources a variant's kernels are built from: a stored DRAM traffic figure holds
+    only while they are unchanged."""
     import hashlib
     h = hashlib.sha1()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_SOURCES[variant]:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
@@ -614,7 +617,7 @@ def main():
     achieved = flops / (per_variant[dom] * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     tr = TRAFFIC.get(dom)
-    traffic = tr[0] if tr and tr[1] == kernel_sources_sha() else None
+    traffic = tr[0] if tr and tr[1] == kernel_sources_sha(dom) else None
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": traffic, "kernel": dom,
             "peak_source": f"{peak_src} bf16 burst", "ms_per_launch": per_variant[dom]}

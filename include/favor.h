@@ -78,10 +78,15 @@ typedef enum {
 /*
  * bf16 forward pass: the tensor-core path.
  * q, k, v, omega, out: device pointers to __nv_bfloat16, 16-byte aligned, layouts above.
- * Supported: d in {16, 32, 64, 128}; 1 <= M <= 256 (trig) or <= 512 (relu); L >= 1 (ragged
- * tails are masked). Bidirectional with d = 128 needs M <= 128 (shared memory of the query
- * kernel). Causal needs d <= 64 and B*H*ceil(M/64) < 2^31. Other shapes return
- * FAVOR_ERR_UNSUPPORTED and launch nothing.
+ * Tensor-core kernels: d in {16, 32, 64, 128}; 1 <= M <= 256 (trig) or <= 512 (relu); L >= 1
+ * (ragged tails are masked). Bidirectional with d = 128 needs M <= 128 (shared memory of the
+ * query kernel). Causal needs d <= 64 and B*H*ceil(M/64) < 2^31.
+ * Other shapes with 1 <= d <= 128, M <= 512, B*H <= 65535 and ceil(L/64) <= 65535 (for
+ * example causal d = 128, or d = 48) run the fp32 CUDA-core kernels of favor_attention_f32 on
+ * fp32 copies of q, k, v and omega (an exact widening on the device) and round the result to
+ * bf16 once; their scratch (the copies, the fp32 output and the fp32 path's chunk states) comes
+ * from the same pool (favor_workspace_bytes). Shapes beyond that return FAVOR_ERR_UNSUPPORTED
+ * and launch nothing.
  * Launches: bidirectional is three kernels on `stream` (key-side partial states over every SM,
  * their merge into per-head state images, then the queries); its scratch comes from the
  * library's stream-ordered pool and is released on the same stream (favor_workspace_bytes gives
@@ -104,7 +109,8 @@ int favor_attention(const void* q, const void* k, const void* v, const void* ome
 /*
  * As favor_attention, with an explicit causal chunk length. The chunk changes how the prefix
  * sum is blocked, not its value. The tensor-core kernel scans 128-token chunks: chunk 0 (the
- * default) or 128; any other value returns FAVOR_ERR_UNSUPPORTED when causal != 0. Ignored when
+ * default) or 128; any other value returns FAVOR_ERR_UNSUPPORTED when causal != 0, and so does
+ * any chunk but 0 for a shape on the CUDA-core route (which blocks by 64 tokens). Ignored when
  * causal == 0.
  */
 int favor_attention_chunked(const void* q, const void* k, const void* v, const void* omega,
@@ -284,7 +290,8 @@ int favor_selftest_sincos(const float* u, float* sin_out, float* cos_out, int n,
  * only; no launch). Bidirectional: the key kernel's partial states (fp32) and their references,
  * and the merged state images the query kernel reads; the run split follows the current
  * device's SM count. Causal: 0 (the state stays in TMEM, partial rows cross the cluster in
- * shared memory). 0 for non-positive sizes and for shapes without a kernel.
+ * shared memory). Shapes on the CUDA-core route: the fp32 copies of q, k, v, out and omega plus
+ * the fp32 path's chunk states. 0 for non-positive sizes and for shapes without a kernel.
  */
 size_t favor_workspace_bytes(int B, int H, int L, int d, int M, int feature_kind, int causal);
 

@@ -122,7 +122,9 @@ def _check_out(out, like, name="out"):
 
 def favor_attention(q, k, v, omega, out=None, feature_kind=FAVOR_TRIG, causal=False, chunk=0,
                     stream=None):
-    """bf16 FAVOR forward on the tensor-core path. q, k, v: [B,H,L,d]; omega: [H,M,d]."""
+    """bf16 FAVOR forward. q, k, v: [B,H,L,d]; omega: [H,M,d]. Tensor-core kernels for the shapes
+    they cover; other shapes up to d = 128, M = 512 run the fp32 CUDA-core kernels on widened
+    copies (favor_attention in include/favor.h)."""
     import torch
     B, H, L, d, M = _check_qkv(q, k, v, omega, torch.bfloat16)
     if out is None:

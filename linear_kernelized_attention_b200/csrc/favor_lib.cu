@@ -281,7 +281,7 @@ int launch_split_t(const SplitPlan& pl, const void* q, const void* k, const void
   {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)pl.npairs, bs::StateCfg<KIND, DP>::R / 32, 1);
-    cfg.blockDim = dim3(256, 1, 1);
+    cfg.blockDim = dim3(bs::merge_threads<KIND, DP>(), 1, 1);
     cfg.stream = st;
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
@@ -378,6 +378,46 @@ int launch_causal_fs(const void* q, const void* k, const void* v, const void* om
 }
 
 // ------------------------------------------------------------------ fp32 path
+}  // namespace
+
+namespace favor {
+namespace cvt {
+// bf16 -> fp32 (exact) and fp32 -> bf16 (round to nearest even) over a flat array; x and y are
+// 16-byte aligned, eight elements per step, then the tail one by one.
+__global__ void __launch_bounds__(256) k_widen(const __nv_bfloat16* __restrict__ x, float* __restrict__ y,
+                                               long long n) {
+  const long long n8 = n / 8, stride = (long long)gridDim.x * blockDim.x;
+  const long long t0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  for (long long i = t0; i < n8; i += stride) {
+    const uint4 w = reinterpret_cast<const uint4*>(x)[i];
+    const float4 a = make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u),
+                                 __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u));
+    const float4 b = make_float4(__uint_as_float(w.z << 16), __uint_as_float(w.z & 0xFFFF0000u),
+                                 __uint_as_float(w.w << 16), __uint_as_float(w.w & 0xFFFF0000u));
+    reinterpret_cast<float4*>(y)[2 * i] = a;
+    reinterpret_cast<float4*>(y)[2 * i + 1] = b;
+  }
+  for (long long i = 8 * n8 + t0; i < n; i += stride) y[i] = __bfloat162float(x[i]);
+}
+
+__global__ void __launch_bounds__(256) k_narrow(const float* __restrict__ y, __nv_bfloat16* __restrict__ x,
+                                                long long n) {
+  const long long n8 = n / 8, stride = (long long)gridDim.x * blockDim.x;
+  const long long t0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  for (long long i = t0; i < n8; i += stride) {
+    const float4 a = reinterpret_cast<const float4*>(y)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(y)[2 * i + 1];
+    reinterpret_cast<uint4*>(x)[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                                                pack_bf16x2(b.z, b.w));
+  }
+  for (long long i = 8 * n8 + t0; i < n; i += stride) x[i] = __float2bfloat16_rn(y[i]);
+}
+}  // namespace cvt
+}  // namespace favor
+
+namespace {
+using namespace favor;
+
 size_t f32_workspace(int BH, int L, int d, int M, int kind) {
   const int F = kind == FAVOR_TRIG ? 2 * M : M;
   const int nch = (L + f32::kChunk - 1) / f32::kChunk;
@@ -411,6 +451,54 @@ int launch_f32(const float* q, const float* k, const float* v, const float* omeg
     f32::k_scan_chunks<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(dS, nch, per_chunk, total, causal);
     f32::k_output<<<dim3(nch, BH), f32::kThreads, sm_out, st>>>(q, k, v, omega, cmax, dS, out, H, L, d, M,
                                                                 F, kind, causal);
+    if (cudaGetLastError() != cudaSuccess) rc = FAVOR_ERR_CUDA;
+  }
+  cudaFreeAsync(ws, st);
+  return rc;
+}
+
+// ------------------------------------------------------------------ bf16 shapes the tensor-core kernels leave out
+// Causal d > 64, bidirectional trig d = 128 with M > 128, d outside {16, 32, 64, 128} and trig
+// 256 < M <= 512 run the fp32 CUDA-core kernels on fp32 copies of the bf16 inputs (the widening is
+// exact) and round the result to bf16 once. Scratch: the four fp32 copies and the fp32 output, then
+// the fp32 path's own scratch, both from the stream-ordered pool.
+size_t round_up256(size_t b) { return (b + 255) / 256 * 256; }
+
+bool cuda_core_route_ok(long long BH, int L, int d, int M) {
+  return d <= f32::kMaxD && M <= 512 && BH <= 65535 && (L + f32::kChunk - 1) / f32::kChunk <= 65535;
+}
+
+size_t cuda_core_route_bytes(long long BH, int H, int L, int d, int M) {
+  const size_t n = (size_t)BH * L * d;
+  return 4 * round_up256(n * sizeof(float)) + round_up256((size_t)H * M * d * sizeof(float));
+}
+
+int launch_bf16_cuda_cores(const void* q, const void* k, const void* v, const void* omega, void* out, int B, int H,
+                           int L, int d, int M, int kind, int causal, cudaStream_t st) {
+  const long long BH = (long long)B * H;
+  if (!cuda_core_route_ok(BH, L, d, M)) return FAVOR_ERR_UNSUPPORTED;
+  const long long n = BH * L * d, nom = (long long)H * M * d;
+  void* ws = nullptr;
+  int rc = scratch_alloc(&ws, cuda_core_route_bytes(BH, H, L, d, M), st);
+  if (rc != FAVOR_OK) return rc;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  const size_t nb = round_up256((size_t)n * sizeof(float));
+  float* qf = reinterpret_cast<float*>(w8);
+  float* kf = reinterpret_cast<float*>(w8 + nb);
+  float* vf = reinterpret_cast<float*>(w8 + 2 * nb);
+  float* of = reinterpret_cast<float*>(w8 + 3 * nb);
+  float* omf = reinterpret_cast<float*>(w8 + 4 * nb);
+  auto grid = [](long long m) {
+    return (unsigned)std::max<long long>(1, std::min<long long>((m / 8 + 255) / 256, 148ll * 16));
+  };
+  cvt::k_widen<<<grid(n), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), qf, n);
+  cvt::k_widen<<<grid(n), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(k), kf, n);
+  cvt::k_widen<<<grid(n), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(v), vf, n);
+  cvt::k_widen<<<grid(nom), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(omega), omf, nom);
+  rc = cudaGetLastError() == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
+  if (rc == FAVOR_OK) rc = launch_f32(qf, kf, vf, omf, of, B, H, L, d, M, kind, causal, st);
+  if (rc == FAVOR_OK) {
+    cvt::k_narrow<<<grid(n), 256, 0, st>>>(of, static_cast<__nv_bfloat16*>(out), n);
     if (cudaGetLastError() != cudaSuccess) rc = FAVOR_ERR_CUDA;
   }
   cudaFreeAsync(ws, st);
@@ -607,12 +695,16 @@ size_t favor_workspace_bytes(int B, int H, int L, int d, int M, int feature_kind
   if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || M <= 0) return 0;
   if ((long long)B * H > INT_MAX) return 0;
   if (feature_kind != FAVOR_TRIG && feature_kind != FAVOR_RELU) return 0;
-  if (check_tc_shape(d, M, feature_kind, causal) != FAVOR_OK) return 0;
-  // causal: the state stays in TMEM and partial rows cross the cluster in shared memory
-  if (causal) return 0;
-  SplitPlan pl{};
-  if (!plan_split(pl, B * H, L, d, M, feature_kind)) return 0;
-  return pl.ws_bytes;
+  const long long BH = (long long)B * H;
+  if (check_tc_shape(d, M, feature_kind, causal) == FAVOR_OK) {
+    // causal: the state stays in TMEM and partial rows cross the cluster in shared memory
+    if (causal) return 0;
+    SplitPlan pl{};
+    if (plan_split(pl, (int)BH, L, d, M, feature_kind)) return pl.ws_bytes;
+  }
+  if (!cuda_core_route_ok(BH, L, d, M)) return 0;
+  // the CUDA-core route: fp32 copies and output, then (not at the same time) the fp32 path's scratch
+  return cuda_core_route_bytes(BH, H, L, d, M) + f32_workspace((int)BH, L, d, M, feature_kind);
 }
 
 int favor_attention_chunked(const void* q, const void* k, const void* v, const void* omega,
@@ -621,13 +713,18 @@ int favor_attention_chunked(const void* q, const void* k, const void* v, const v
   int rc = check_common(q, k, v, omega, out, B, H, L, d, M, feature_kind);
   if (rc != FAVOR_OK) return rc;
   if ((rc = check_device()) != FAVOR_OK) return rc;
-  if ((rc = check_tc_shape(d, M, feature_kind, causal)) != FAVOR_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (causal) {
-    if (chunk != 0 && chunk != cf::kTile) return FAVOR_ERR_UNSUPPORTED;
-    return launch_causal_fs(q, k, v, omega, out, B, H, L, d, M, feature_kind, st);
+  if (check_tc_shape(d, M, feature_kind, causal) == FAVOR_OK) {
+    if (causal) {
+      if (chunk != 0 && chunk != cf::kTile) return FAVOR_ERR_UNSUPPORTED;
+      return launch_causal_fs(q, k, v, omega, out, B, H, L, d, M, feature_kind, st);
+    }
+    rc = launch_bidir_split(q, k, v, omega, out, B, H, L, d, M, feature_kind, st);
+    if (rc != FAVOR_ERR_UNSUPPORTED) return rc;  // unsupported: no shared-memory plan, nothing launched
   }
-  return launch_bidir_split(q, k, v, omega, out, B, H, L, d, M, feature_kind, st);
+  // shapes the tensor-core kernels leave out: the fp32 CUDA-core kernels on widened copies
+  if (causal && chunk != 0) return FAVOR_ERR_UNSUPPORTED;
+  return launch_bf16_cuda_cores(q, k, v, omega, out, B, H, L, d, M, feature_kind, causal, st);
 }
 
 int favor_attention(const void* q, const void* k, const void* v, const void* omega, void* out,

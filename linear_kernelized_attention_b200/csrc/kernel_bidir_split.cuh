@@ -552,15 +552,30 @@ __device__ __forceinline__ uint32_t img_byte(int f, int n) {
          uint32_t(f & 7) * 2;
 }
 
-// One block per (pair, 32 state rows). Trig feature order within a 128-angle block: 32-angle
-// groups of [cos 32 | sin 32], matching the query kernel's packing. The first warp turns the
-// head's slot metadata into per-slot weights in shared memory; then every thread sums its
-// elements over the pair's slots with all loads of an element in flight together.
+// One block per (pair, 32 state rows), one thread per 8-row work item (4 (d_pad + 16) threads).
+// Trig feature order within a 128-angle block: 32-angle groups of [cos 32 | sin 32], matching the
+// query kernel's packing. The first warp turns the head's slot metadata into per-slot weights in
+// shared memory while every thread's loads of its first slots are in flight; then every thread
+// sums its item over the pair's slots.
 constexpr int kMergeMaxSlots = 64;  // slots of one head (nab * smax) the merge can weight
 
 template <int KIND, int DP>
-__global__ void __launch_bounds__(256) k_bidir_merge(const MergeParams p) {
+__host__ __device__ constexpr int merge_threads() { return 4 * (DP + 16); }  // one 8-row work item per thread
+
+// Blocks per SM the merge is compiled for, and the slots of a work item whose loads are issued
+// before the weights are known: trig has twice the blocks of ReLU (256 state rows per pair, not
+// 128), so it keeps fewer loads in flight per thread to fit four blocks per SM (one wave at the
+// usual shapes); ReLU fits two blocks per SM with four.
+template <int KIND>
+__host__ __device__ constexpr int merge_min_blocks() { return KIND == 0 ? 4 : 2; }
+template <int KIND>
+__host__ __device__ constexpr int merge_pre() { return KIND == 0 ? 2 : 4; }
+
+template <int KIND, int DP>
+__global__ void __launch_bounds__(merge_threads<KIND, DP>(), merge_min_blocks<KIND>())
+    k_bidir_merge(const MergeParams p) {
   constexpr int NV = DP + 16, R = KIND == 0 ? 256 : 128, FB = R;
+  constexpr int kMergePre = merge_pre<KIND>();
   __shared__ float wts[kMergeMaxSlots];
   __shared__ float scale_s;
   pdl_launch_dependents();  // the query kernel may start its projections
@@ -569,24 +584,29 @@ __global__ void __launch_bounds__(256) k_bidir_merge(const MergeParams p) {
   const int rb = blockIdx.y;
   const long long bh = pr / p.nab;
   const int ab = (int)(pr % p.nab);
-  const int ns = min(nslots(pr, p), kMergeMaxSlots);
+  // slot counts of the head's (at most 4) angle blocks: lane a of every warp evaluates block a's
+  // (two 64-bit divisions), and the warp shares them
+  const int nsl = (threadIdx.x & 31) < p.nab ? nslots(bh * p.nab + (threadIdx.x & 31), p) : 0;
+  const int ns = min(__shfl_sync(0xffffffffu, nsl, ab), kMergeMaxSlots);
   uint8_t* img = p.img + bh * p.img_bytes;
   const float* part = p.part + pr * p.smax * (long long)(DP + 1) * R;
   const long long sstride = (long long)(DP + 1) * R;
-  // The partial states do not depend on the weights: every thread starts loading slots 0 and 1
-  // of its first work item before the first warp has turned the metadata into weights.
-  const int w0 = threadIdx.x;
-  const bool pre = w0 < 4 * NV && (w0 >> 2) <= DP;
-  float4 pa0 = make_float4(0.f, 0.f, 0.f, 0.f), pa1 = pa0, pb0 = pa0, pb1 = pa0;
-  if (pre) {
-    const float* src = part + (long long)(w0 >> 2) * R + rb * 32 + (w0 & 3) * 8;
-    if (ns > 0) {
-      pa0 = *reinterpret_cast<const float4*>(src);
-      pa1 = *reinterpret_cast<const float4*>(src + 4);
-    }
-    if (ns > 1) {
-      pb0 = *reinterpret_cast<const float4*>(src + sstride);
-      pb1 = *reinterpret_cast<const float4*>(src + sstride + 4);
+  // Work item of this thread: 8 consecutive state rows of value row nn (two float4 loads per
+  // slot), i.e. 8 consecutive features of the image, one 16-byte chunk. The partial states do not
+  // depend on the weights: the loads of the first kMergePre slots are issued before the first
+  // warp has turned the metadata into weights, so they are in flight together with its loads.
+  const int w = threadIdx.x, oct = w & 3, nn = w >> 2;
+  const int r0 = rb * 32 + oct * 8;
+  const bool live = nn <= DP;
+  const float* src = part + (long long)nn * R + r0;
+  float4 pre[kMergePre][2];
+#pragma unroll
+  for (int s = 0; s < kMergePre; ++s) {
+    pre[s][0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    pre[s][1] = pre[s][0];
+    if (live && s < ns) {
+      pre[s][0] = *reinterpret_cast<const float4*>(src + s * sstride);
+      pre[s][1] = *reinterpret_cast<const float4*>(src + s * sstride + 4);
     }
   }
   if (threadIdx.x < 32) {
@@ -600,9 +620,10 @@ __global__ void __launch_bounds__(256) k_bidir_merge(const MergeParams p) {
       const int a2 = e >> 1, sl = lane + 32 * (e & 1);
       mc[e] = -INFINITY;
       mb[e] = 0.f;
+      const int ns2 = __shfl_sync(0xffffffffu, nsl, a2 & 3);
       if (a2 < p.nab) {
         const long long q2 = bh * p.nab + a2;
-        if (sl < nslots(q2, p)) {
+        if (sl < ns2) {
           const float* m = p.meta + (q2 * p.smax + sl) * 2;
           mc[e] = KIND == 0 ? m[0] : 0.f;
           mb[e] = m[1];
@@ -617,9 +638,9 @@ __global__ void __launch_bounds__(256) k_bidir_merge(const MergeParams p) {
     for (int e = 0; e < 8; ++e) {
       const int a2 = e >> 1, sl = lane + 32 * (e & 1);
       if (mc[e] == -INFINITY) continue;
-      const float w = KIND == 0 ? __expf(mc[e] - cmax) : 1.f;
-      bound += w * mb[e];
-      if (a2 == ab) wts[sl] = w;
+      const float wt = KIND == 0 ? __expf(mc[e] - cmax) : 1.f;
+      bound += wt * mb[e];
+      if (a2 == ab) wts[sl] = wt;
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) bound += __shfl_xor_sync(0xffffffffu, bound, o);
@@ -627,68 +648,46 @@ __global__ void __launch_bounds__(256) k_bidir_merge(const MergeParams p) {
   }
   __syncthreads();
   const float scale = scale_s;
-  // one work item = 8 consecutive state rows of one value row: two float4 loads per slot, and 8
-  // consecutive features of the image, i.e. one 16-byte chunk
-  for (int w = threadIdx.x; w < 4 * NV; w += blockDim.x) {
-    const int oct = w & 3, nn = w >> 2;
-    const int r0 = rb * 32 + oct * 8;
-    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (nn <= DP) {
-      const float* src = part + (long long)nn * R + r0;
-      int s = 0;
-      if (w == w0) {
-        // slots 0 and 1, loaded before the weights were known
-        const float wa = ns > 0 ? wts[0] : 0.f, wb = ns > 1 ? wts[1] : 0.f;
-        v[0] = fmaf(wa, pa0.x, wb * pb0.x);
-        v[1] = fmaf(wa, pa0.y, wb * pb0.y);
-        v[2] = fmaf(wa, pa0.z, wb * pb0.z);
-        v[3] = fmaf(wa, pa0.w, wb * pb0.w);
-        v[4] = fmaf(wa, pa1.x, wb * pb1.x);
-        v[5] = fmaf(wa, pa1.y, wb * pb1.y);
-        v[6] = fmaf(wa, pa1.z, wb * pb1.z);
-        v[7] = fmaf(wa, pa1.w, wb * pb1.w);
-        s = min(ns, 2);
-      }
-      for (; s + 2 <= ns; s += 2) {
-        const float4 a0 = *reinterpret_cast<const float4*>(src + s * sstride);
-        const float4 a1 = *reinterpret_cast<const float4*>(src + s * sstride + 4);
-        const float4 b0 = *reinterpret_cast<const float4*>(src + (s + 1) * sstride);
-        const float4 b1 = *reinterpret_cast<const float4*>(src + (s + 1) * sstride + 4);
-        const float wa = wts[s], wb = wts[s + 1];
-        v[0] = fmaf(wa, a0.x, fmaf(wb, b0.x, v[0]));
-        v[1] = fmaf(wa, a0.y, fmaf(wb, b0.y, v[1]));
-        v[2] = fmaf(wa, a0.z, fmaf(wb, b0.z, v[2]));
-        v[3] = fmaf(wa, a0.w, fmaf(wb, b0.w, v[3]));
-        v[4] = fmaf(wa, a1.x, fmaf(wb, b1.x, v[4]));
-        v[5] = fmaf(wa, a1.y, fmaf(wb, b1.y, v[5]));
-        v[6] = fmaf(wa, a1.z, fmaf(wb, b1.z, v[6]));
-        v[7] = fmaf(wa, a1.w, fmaf(wb, b1.w, v[7]));
-      }
-      if (s < ns) {
-        const float4 a0 = *reinterpret_cast<const float4*>(src + s * sstride);
-        const float4 a1 = *reinterpret_cast<const float4*>(src + s * sstride + 4);
-        const float wa = wts[s];
-        v[0] = fmaf(wa, a0.x, v[0]);
-        v[1] = fmaf(wa, a0.y, v[1]);
-        v[2] = fmaf(wa, a0.z, v[2]);
-        v[3] = fmaf(wa, a0.w, v[3]);
-        v[4] = fmaf(wa, a1.x, v[4]);
-        v[5] = fmaf(wa, a1.y, v[5]);
-        v[6] = fmaf(wa, a1.z, v[6]);
-        v[7] = fmaf(wa, a1.w, v[7]);
-      }
-    }
-    const int a0 = KIND == 0 ? (r0 & 127) : r0;  // first angle of the octet (same sin/cos block)
-    uint32_t pk[4];
+  float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (live) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float x0 = ab * 128 + a0 + 2 * e < p.M ? v[2 * e] : 0.f;      // padded angles read as zero
-      const float x1 = ab * 128 + a0 + 2 * e + 1 < p.M ? v[2 * e + 1] : 0.f;
-      pk[e] = KIND == 0 ? pack_f16x2(x0 * scale, x1 * scale) : pack_bf16x2(x0, x1);
+    for (int s = 0; s < kMergePre; ++s) {
+      if (s < ns) {
+        const float wa = wts[s];
+        v[0] = fmaf(wa, pre[s][0].x, v[0]);
+        v[1] = fmaf(wa, pre[s][0].y, v[1]);
+        v[2] = fmaf(wa, pre[s][0].z, v[2]);
+        v[3] = fmaf(wa, pre[s][0].w, v[3]);
+        v[4] = fmaf(wa, pre[s][1].x, v[4]);
+        v[5] = fmaf(wa, pre[s][1].y, v[5]);
+        v[6] = fmaf(wa, pre[s][1].z, v[6]);
+        v[7] = fmaf(wa, pre[s][1].w, v[7]);
+      }
     }
-    const int f0 = KIND == 0 ? ab * FB + (a0 >> 5) * 64 + (r0 >> 7) * 32 + (a0 & 31) : ab * FB + r0;
-    *reinterpret_cast<uint4*>(img + img_byte<NV>(f0, nn)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    for (int s = kMergePre; s < ns; ++s) {
+      const float4 a0 = *reinterpret_cast<const float4*>(src + s * sstride);
+      const float4 a1 = *reinterpret_cast<const float4*>(src + s * sstride + 4);
+      const float wa = wts[s];
+      v[0] = fmaf(wa, a0.x, v[0]);
+      v[1] = fmaf(wa, a0.y, v[1]);
+      v[2] = fmaf(wa, a0.z, v[2]);
+      v[3] = fmaf(wa, a0.w, v[3]);
+      v[4] = fmaf(wa, a1.x, v[4]);
+      v[5] = fmaf(wa, a1.y, v[5]);
+      v[6] = fmaf(wa, a1.z, v[6]);
+      v[7] = fmaf(wa, a1.w, v[7]);
+    }
   }
+  const int a0 = KIND == 0 ? (r0 & 127) : r0;  // first angle of the octet (same sin/cos block)
+  uint32_t pk[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float x0 = ab * 128 + a0 + 2 * e < p.M ? v[2 * e] : 0.f;      // padded angles read as zero
+    const float x1 = ab * 128 + a0 + 2 * e + 1 < p.M ? v[2 * e + 1] : 0.f;
+    pk[e] = KIND == 0 ? pack_f16x2(x0 * scale, x1 * scale) : pack_bf16x2(x0, x1);
+  }
+  const int f0 = KIND == 0 ? ab * FB + (a0 >> 5) * 64 + (r0 >> 7) * 32 + (a0 & 31) : ab * FB + r0;
+  *reinterpret_cast<uint4*>(img + img_byte<NV>(f0, nn)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
 }
 
 // ============================================================================ queries
@@ -715,13 +714,16 @@ struct QueryParams {
 struct alignas(16) QueryMisc {
   int abort_flag;
   uint32_t tmem_base;
-  uint64_t head_full, head_free;
+  uint64_t om_full;    // a head's Omega blocks (the projections)
+  uint64_t head_full;  // a head's state image (the state products)
+  uint64_t head_free;  // both buffers may take the next head
   uint64_t q_full[2], q_empty[2];
   uint64_t u_full[3], p_full[3], buf_free[3];
   uint64_t num_full[2], num_empty[2];
   uint64_t drain;
   uint64_t out_sync;  // bounded barrier among the 128 output threads
 };
+static_assert(sizeof(QueryMisc) <= 1024, "misc block");
 
 template <int KIND, int DP>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -748,6 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     ms->abort_flag = 0;
+    mbar_init(bar(ms->om_full), 1);
     mbar_init(bar(ms->head_full), 1);
     mbar_init(bar(ms->head_free), 1);
     for (int i = 0; i < 2; ++i) {
@@ -799,15 +802,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued = t + 1;
         if (w.first()) {
           const int hk = w.k;
-          if (hk == 0) pdl_wait();  // the merge has written the state images
           if (hk >= 1 && !mbar_wait(bar(ms->head_free), (hk - 1) & 1, abort_flag)) break;
           const int h = (int)(bh % p.H);
           const uint8_t* src = p.img + bh * p.img_bytes;
-          if (leader) {
-            mbar_arrive_expect_tx(bar(ms->head_full), p.om_bytes + p.img_bytes);
+          if (leader) {  // Omega does not come from the merge: the projections may start now
+            mbar_arrive_expect_tx(bar(ms->om_full), p.om_bytes);
             for (int ab = 0; ab < nab; ++ab)
               for (int kb = 0; kb < NCB; ++kb)
-                tma_load_3d(s_om + (ab * NCB + kb) * kBoxB, &tm_om, bar(ms->head_full), kb * 64, ab * 128, h);
+                tma_load_3d(s_om + (ab * NCB + kb) * kBoxB, &tm_om, bar(ms->om_full), kb * 64, ab * 128, h);
+          }
+          if (hk == 0) pdl_wait();  // the merge has written the state images
+          if (leader) {
+            mbar_arrive_expect_tx(bar(ms->head_full), p.img_bytes);
             for (int off = 0; off < p.img_bytes; off += 32768) {
               const int sz = min(32768, p.img_bytes - off);
               bulk_load(s_img + off, src + off, sz, bar(ms->head_full));
@@ -820,7 +826,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr long long kDrain = kWaitLimitCycles / 8;
         for (int t = issued > 2 ? issued - 2 : 0; t < issued; ++t)
           mbar_wait(bar(ms->q_full[t & 1]), (t >> 1) & 1, nullptr, kDrain);
-        if (heads > 0) mbar_wait(bar(ms->head_full), (heads - 1) & 1, nullptr, kDrain);
+        if (heads > 0) {
+          mbar_wait(bar(ms->om_full), (heads - 1) & 1, nullptr, kDrain);
+          mbar_wait(bar(ms->head_full), (heads - 1) & 1, nullptr, kDrain);
+        }
       }
     }
     __syncwarp();
@@ -839,7 +848,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         w1.advance_to(t);
         if (ab == 0) {
           if (!mbar_wait(bar(ms->q_full[s]), (t >> 1) & 1, abort_flag)) break;
-          if (w1.first() && !mbar_wait(bar(ms->head_full), w1.k & 1, abort_flag)) break;
+          if (w1.first() && !mbar_wait(bar(ms->om_full), w1.k & 1, abort_flag)) break;
         }
         if (j >= NBQ && !mbar_wait(bar(ms->buf_free[b]), ((j - NBQ) / NBQ) & 1, abort_flag)) break;
         tc_fence_after();
@@ -873,6 +882,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t = j / nab, ab = j - t * nab, b = j % NBQ, nb = t % NBN;
         w2.advance_to(t);
         if (!(ok = mbar_wait(bar(ms->p_full[b]), (j / NBQ) & 1, abort_flag))) break;
+        if (ab == 0 && w2.first() && !(ok = mbar_wait(bar(ms->head_full), w2.k & 1, abort_flag))) break;
         if (ab == 0 && t >= NBN && !(ok = mbar_wait(bar(ms->num_empty[nb]), ((t / NBN) - 1) & 1, abort_flag))) break;
         tc_fence_after();
         const uint32_t dn = tmem + C::kNumCol + nb * NV;

@@ -75,14 +75,20 @@ def test_workspace_bytes_is_host_only():
     assert F.favor_workspace_bytes(1, 1, 1, 64, 64, 0, False) >= 0
     assert F.favor_workspace_bytes(0, 1, 1, 64, 64, 0, False) == 0
     # bidirectional: at least one fp32 partial state per (head, 128-angle block) and one state
-    # image per head; causal takes none; unsupported shapes take none
+    # image per head; causal takes none
     B, H, L, d, M = 4, 8, 4096, 64, 256
     ws = F.favor_workspace_bytes(B, H, L, d, M, 0, False)
     assert ws >= B * H * 2 * (d + 1) * 256 * 4 + B * H * 2 * 256 * (d + 16) * 2
     assert F.favor_workspace_bytes(B, H, L, d, M, 1, False) > 0
     assert F.favor_workspace_bytes(B, H, L, d, M, 0, True) == 0
-    assert F.favor_workspace_bytes(B, H, L, 48, M, 0, False) == 0
-    assert F.favor_workspace_bytes(B, H, L, d, 272, 0, False) == 0
+    # shapes the tensor-core kernels leave out take the CUDA-core route: fp32 copies of q, k, v,
+    # the output and Omega, plus the fp32 path's chunk states
+    for (dd, MM, causal) in [(48, M, False), (d, 272, False), (128, M, True), (128, M, False)]:
+        n = B * H * L * dd
+        assert F.favor_workspace_bytes(B, H, L, dd, MM, 0, causal) >= 4 * 4 * n + 4 * H * MM * dd
+    # beyond every kernel: none
+    assert F.favor_workspace_bytes(B, H, L, 136, M, 0, False) == 0
+    assert F.favor_workspace_bytes(B, H, L, d, 528, 1, True) == 0
 
 
 # ------------------------------------------------------------------ decode entry points

@@ -129,9 +129,9 @@ def test_bidir_head_sizes(kind, d, M):
 def test_bidir_unsupported_shapes_are_refused():
     import torch
     import linear_kernelized_attention_b200 as F
-    # d = 128 with trig M = 256: the state image (512 features x 144 rows) and the operand tiles do
-    # not fit in one CTA's shared memory; d = 48 is not a supported head size
-    for (d, M, kind) in ((128, 256, 0), (48, 64, 0)):
+    # beyond every kernel: d > 128, or M > 512. (d = 128 with trig M = 256, whose state image and
+    # operand tiles do not fit one CTA's shared memory, and d = 48 take the CUDA-core route.)
+    for (d, M, kind) in ((136, 64, 0), (64, 528, 1)):
         q = torch.zeros((1, 1, 128, d), dtype=torch.bfloat16, device="cuda")
         om = torch.zeros((1, M, d), dtype=torch.bfloat16, device="cuda")
         with pytest.raises(F.FavorError) as e:
