@@ -265,11 +265,19 @@ __global__ void __launch_bounds__(kThreads)
 // constrains the directions to a random subsample of an orthogonal matrix.
 //
 // Rows go in panels of kOrfPanel. A panel is first made orthogonal to every finished row by two
-// passes of block classical Gram-Schmidt (one warp per panel row, no block barrier), then
+// passes of block classical Gram-Schmidt (8x8x4 fp64 tensor-core products), then
 // orthonormalised within itself by two passes of Cholesky QR on its Gram matrix (the lower
 // Cholesky factor L of V V^T gives V <- L^-1 V). Both are exact reformulations of Gram-Schmidt in
 // order (the same Q), in fp64; the serial chain is a few dozen small steps per panel instead of a
 // block-wide reduction per row.
+// D = A B + D on the fp64 tensor cores, 8x8x4: lane l holds A[l/4][l%4], B[l%4][l/4] and
+// D[l/4][2(l%4)], D[l/4][2(l%4)+1].
+__device__ __forceinline__ void mma_f64_m8n8k4(double& d0, double& d1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(d0), "+d"(d1)
+               : "d"(a), "d"(b));
+}
+
 constexpr int kOrfThreads = 512;
 constexpr int kOrfPanel = 8;  // rows per panel: one warp each
 
@@ -341,51 +349,44 @@ __global__ void __launch_bounds__(kOrfThreads)
     const int nr = min(kOrfPanel, d - r0);
     const bool act = warp < nr;
     double* vi = sq + (size_t)(r0 + warp) * ld;
-    // (1) two passes of classical Gram-Schmidt of panel row r0 + warp against rows 0 .. r0-1:
-    // lane l forms the coefficients of rows l, l+32, l+64, l+96, then owns columns l + 32 e
-    if (act && r0 > 0) {
-      const int nm = (r0 + 31) >> 5;  // warp-uniform
-      double* cw = coef + warp * 128;
+    // (1) two passes of block classical Gram-Schmidt of the panel against rows 0 .. r0-1, on the
+    // fp64 tensor cores (mma m8n8k4: the panel is the 8-row side): C = V Q^T over 8-row blocks of
+    // Q, one block per warp, then V -= C Q over 8-column blocks of V, one block per warp
+    if (r0 > 0) {
+      const int gi = lane >> 2, gk = lane & 3, nw = blockDim.x >> 5;
+      const double* arow = sq + (size_t)(r0 + min(gi, nr - 1)) * ld;
       for (int pass = 0; pass < 2; ++pass) {
-        double c[4] = {0.0, 0.0, 0.0, 0.0}, c2[4] = {0.0, 0.0, 0.0, 0.0};
-        const double* qr[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) qr[m] = sq + (size_t)min(lane + 32 * m, r0 - 1) * ld;
-        int t = 0;
-        for (; t + 1 < d; t += 2) {
-          const double x = vi[t], y = vi[t + 1];
-#pragma unroll
-          for (int m = 0; m < 4; ++m)
-            if (m < nm) {
-              c[m] = fma(qr[m][t], x, c[m]);
-              c2[m] = fma(qr[m][t + 1], y, c2[m]);
-            }
+        for (int jb = warp; jb < (r0 >> 3); jb += nw) {
+          double c0 = 0.0, c1 = 0.0;
+          const double* brow = sq + (size_t)(jb * 8 + gi) * ld;
+          for (int t0 = 0; t0 < d; t0 += 4) {
+            const int t = t0 + gk;
+            const double a = (gi < nr && t < d) ? arow[t] : 0.0;
+            const double b = t < d ? brow[t] : 0.0;
+            mma_f64_m8n8k4(c0, c1, a, b);
+          }
+          if (gi < nr) {
+            coef[gi * 128 + jb * 8 + 2 * gk] = c0;
+            coef[gi * 128 + jb * 8 + 2 * gk + 1] = c1;
+          }
         }
-        if (t < d) {
-          const double x = vi[t];
-#pragma unroll
-          for (int m = 0; m < 4; ++m)
-            if (m < nm) c[m] = fma(qr[m][t], x, c[m]);
+        __syncthreads();
+        for (int tb = warp; tb < ((d + 7) >> 3); tb += nw) {
+          double d0 = 0.0, d1 = 0.0;
+          const int tn = tb * 8 + gi;
+          for (int j0 = 0; j0 < r0; j0 += 4) {
+            const double a = gi < nr ? coef[gi * 128 + j0 + gk] : 0.0;
+            const double b = tn < d ? sq[(size_t)(j0 + gk) * ld + tn] : 0.0;
+            mma_f64_m8n8k4(d0, d1, a, b);
+          }
+          const int t = tb * 8 + 2 * gk;
+          if (gi < nr) {
+            double* v = sq + (size_t)(r0 + gi) * ld;
+            if (t < d) v[t] -= d0;
+            if (t + 1 < d) v[t + 1] -= d1;
+          }
         }
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-          if (lane + 32 * m < r0) cw[lane + 32 * m] = c[m] + c2[m];
-        __syncwarp();
-        double a[4] = {0.0, 0.0, 0.0, 0.0}, a2[4] = {0.0, 0.0, 0.0, 0.0};
-        for (int j = 0; j < r0; j += 2) {  // r0 is a multiple of the panel height, so even
-          const double cj = cw[j], ck = cw[j + 1];
-          const double* qj = sq + (size_t)j * ld;
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (lane + 32 * e < d) {
-              a[e] = fma(cj, qj[lane + 32 * e], a[e]);
-              a2[e] = fma(ck, qj[ld + lane + 32 * e], a2[e]);
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (lane + 32 * e < d) vi[lane + 32 * e] -= a[e] + a2[e];
-        __syncwarp();
+        __syncthreads();
       }
     }
     __syncthreads();
