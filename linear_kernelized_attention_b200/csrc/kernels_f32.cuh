@@ -281,9 +281,13 @@ __device__ __forceinline__ void mma_f64_m8n8k4(double& d0, double& d1, double a,
 constexpr int kOrfThreads = 512;
 constexpr int kOrfPanel = 8;  // rows per panel: one warp each
 
-__host__ __device__ constexpr int orf_ld(int d) { return d | 1; }  // odd stride: conflict-free column reads
+// Row stride of the block in shared memory (doubles): 4 modulo 16, so the 8x4 and 4x8 operand
+// fragments of the fp64 MMAs (lane l reads row l/4, column l%4, or the transpose) fall on distinct
+// banks within each half-warp.
+__host__ __device__ constexpr int orf_ld(int d) { return (d + 11) / 16 * 16 + 4; }
+constexpr int kOrfCoefLd = 132;  // coefficient rows, 4 modulo 16 for the same reason
 __host__ __device__ constexpr size_t orf_smem_bytes(int d) {
-  return ((size_t)d * orf_ld(d) + kOrfPanel * 128 + kOrfPanel * kOrfPanel + kOrfPanel + 128) * sizeof(double);
+  return ((size_t)d * orf_ld(d) + kOrfPanel * kOrfCoefLd + kOrfPanel * kOrfPanel + kOrfPanel + 128) * sizeof(double);
 }
 
 __global__ void __launch_bounds__(kOrfThreads)
@@ -292,8 +296,8 @@ __global__ void __launch_bounds__(kOrfThreads)
   extern __shared__ double orf_sm[];
   const int ld = orf_ld(d);
   double* sq = orf_sm;                            // [d][ld] rows being orthonormalised
-  double* coef = sq + (size_t)d * ld;             // [kOrfPanel][128] coefficients against finished rows
-  double* gram = coef + kOrfPanel * 128;          // [kOrfPanel][kOrfPanel] Gram matrix -> Cholesky factor
+  double* coef = sq + (size_t)d * ld;             // [kOrfPanel][kOrfCoefLd] coefficients against finished rows
+  double* gram = coef + kOrfPanel * kOrfCoefLd;   // [kOrfPanel][kOrfPanel] Gram matrix -> Cholesky factor
   double* rdiag = gram + kOrfPanel * kOrfPanel;   // [kOrfPanel] 1 / L_kk
   double* chi = rdiag + kOrfPanel;                // [128] row lengths
   const int h = blockIdx.y, blk = blockIdx.x, nb = gridDim.x;
@@ -366,8 +370,8 @@ __global__ void __launch_bounds__(kOrfThreads)
             mma_f64_m8n8k4(c0, c1, a, b);
           }
           if (gi < nr) {
-            coef[gi * 128 + jb * 8 + 2 * gk] = c0;
-            coef[gi * 128 + jb * 8 + 2 * gk + 1] = c1;
+            coef[gi * kOrfCoefLd + jb * 8 + 2 * gk] = c0;
+            coef[gi * kOrfCoefLd + jb * 8 + 2 * gk + 1] = c1;
           }
         }
         __syncthreads();
@@ -375,7 +379,7 @@ __global__ void __launch_bounds__(kOrfThreads)
           double d0 = 0.0, d1 = 0.0;
           const int tn = tb * 8 + gi;
           for (int j0 = 0; j0 < r0; j0 += 4) {
-            const double a = gi < nr ? coef[gi * 128 + j0 + gk] : 0.0;
+            const double a = gi < nr ? coef[gi * kOrfCoefLd + j0 + gk] : 0.0;
             const double b = tn < d ? sq[(size_t)(j0 + gk) * ld + tn] : 0.0;
             mma_f64_m8n8k4(d0, d1, a, b);
           }
