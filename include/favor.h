@@ -176,10 +176,14 @@ int favor_philox4x64(uint64_t key, uint64_t first_counter, uint64_t n_blocks, ui
 
 /*
  * Host-buffer convenience entry: q, k, v, omega, out are HOST pointers (pinned memory
- * makes the copies asynchronous). Allocates device buffers with cudaMallocAsync on
- * `stream`, copies in, runs favor_attention (dtype_code 1 = bf16) or favor_attention_f32
- * (dtype_code 0 = float), copies out and frees. It synchronises `stream` before returning,
- * so `out` is ready when it returns FAVOR_OK.
+ * makes the copies asynchronous). Allocates device buffers from the pool on `stream`, copies
+ * in, runs favor_attention (dtype_code 1 = bf16) or favor_attention_f32 (dtype_code 0 =
+ * float), copies out and frees. The batch is cut into up to four slices of whole batch entries
+ * (slice i = entries [B i / S, B (i+1) / S)): slice i's copies in run on a library-owned
+ * stream, its forward pass on `stream` and its copy out on a second library stream, so one
+ * slice's compute and copy out overlap the next slice's copies in; each slice's result equals
+ * the device entry run on that slice alone. It synchronises `stream` before returning, so
+ * `out` is ready when it returns FAVOR_OK.
  */
 int favor_attention_host(const void* q, const void* k, const void* v, const void* omega,
                          void* out, int B, int H, int L, int d, int M, int feature_kind,

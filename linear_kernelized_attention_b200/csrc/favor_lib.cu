@@ -176,6 +176,24 @@ int scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
   return cudaMallocFromPoolAsync(p, bytes, pool, st) == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
 
+// Two non-blocking streams per device for the host-buffer entry's copies in and out, created on
+// first use and kept for the life of the process.
+constexpr int kHostSlices = 4;  // batch slices of the host-buffer entry's copy/compute pipeline
+int copy_streams(cudaStream_t* s_in, cudaStream_t* s_out) {
+  static cudaStream_t streams[64][2] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FAVOR_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return FAVOR_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(mu);
+  for (int i = 0; i < 2; ++i)
+    if (!streams[dev][i] && cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking) != cudaSuccess)
+      return FAVOR_ERR_CUDA;
+  *s_in = streams[dev][0];
+  *s_out = streams[dev][1];
+  return FAVOR_OK;
+}
+
 int check_tc_shape(int d, int M, int kind, int causal) {
   if (d != 16 && d != 32 && d != 64 && d != 128) return FAVOR_ERR_UNSUPPORTED;
   if (kind == FAVOR_TRIG && M > 256) return FAVOR_ERR_UNSUPPORTED;
@@ -793,34 +811,67 @@ int favor_attention_host(const void* q, const void* k, const void* v, const void
   if (dtype_code != 0 && dtype_code != 1) return FAVOR_ERR_UNSUPPORTED;
   if ((rc = check_device()) != FAVOR_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  if ((rc = copy_streams(&s_in, &s_out)) != FAVOR_OK) return rc;
   const size_t es = dtype_code == 1 ? 2 : 4;
-  const size_t nx = (size_t)B * H * L * d * es, nom = (size_t)H * M * d * es;
+  const size_t per_b = (size_t)H * L * d * es;  // one batch entry of q, k, v or out
+  const size_t nx = (size_t)B * per_b, nom = (size_t)H * M * d * es;
+  // Batch slices: slice i's copy in, its forward pass and its copy out run on three streams, so
+  // one slice's compute and copy out overlap the next slice's copy in.
+  const int S = std::min(B, kHostSlices);
   void *dq = nullptr, *dk = nullptr, *dv = nullptr, *dom = nullptr, *dout = nullptr;
-  if ((rc = scratch_alloc(&dq, nx, st)) != FAVOR_OK) return rc;
-  scratch_alloc(&dk, nx, st);
-  scratch_alloc(&dv, nx, st);
-  scratch_alloc(&dom, nom, st);
-  scratch_alloc(&dout, nx, st);
-  if (!dk || !dv || !dom || !dout) rc = FAVOR_ERR_CUDA;
-  if (rc == FAVOR_OK) {
-    if (cudaMemcpyAsync(dq, q, nx, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(dk, k, nx, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(dv, v, nx, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(dom, omega, nom, cudaMemcpyHostToDevice, st) != cudaSuccess)
+  cudaEvent_t ev[2 * kHostSlices + 2] = {};
+  const int nev = 2 * S + 2;
+  for (int e = 0; e < nev; ++e)
+    if (cudaEventCreateWithFlags(&ev[e], cudaEventDisableTiming) != cudaSuccess) rc = FAVOR_ERR_CUDA;
+  if (rc == FAVOR_OK && (rc = scratch_alloc(&dq, nx, st)) == FAVOR_OK) {
+    scratch_alloc(&dk, nx, st);
+    scratch_alloc(&dv, nx, st);
+    scratch_alloc(&dom, nom, st);
+    scratch_alloc(&dout, nx, st);
+    if (!dk || !dv || !dom || !dout) rc = FAVOR_ERR_CUDA;
+  }
+  cudaEvent_t ev_alloc = ev[2 * S], ev_done = ev[2 * S + 1];
+  // the copy streams may touch the buffers only after their allocation on `stream`
+  if (rc == FAVOR_OK && (cudaEventRecord(ev_alloc, st) != cudaSuccess || cudaStreamWaitEvent(s_in, ev_alloc, 0) != cudaSuccess ||
+                         cudaStreamWaitEvent(s_out, ev_alloc, 0) != cudaSuccess))
+    rc = FAVOR_ERR_CUDA;
+  if (rc == FAVOR_OK && cudaMemcpyAsync(dom, omega, nom, cudaMemcpyHostToDevice, s_in) != cudaSuccess) rc = FAVOR_ERR_CUDA;
+  int issued = 0;  // slices whose compute was launched
+  for (int i = 0; rc == FAVOR_OK && i < S; ++i) {
+    const int b0 = (int)((long long)B * i / S), b1 = (int)((long long)B * (i + 1) / S);
+    const size_t off = (size_t)b0 * per_b, len = (size_t)(b1 - b0) * per_b;
+    uint8_t *q8 = static_cast<uint8_t*>(dq) + off, *k8 = static_cast<uint8_t*>(dk) + off,
+            *v8 = static_cast<uint8_t*>(dv) + off, *o8 = static_cast<uint8_t*>(dout) + off;
+    if (cudaMemcpyAsync(q8, static_cast<const uint8_t*>(q) + off, len, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaMemcpyAsync(k8, static_cast<const uint8_t*>(k) + off, len, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaMemcpyAsync(v8, static_cast<const uint8_t*>(v) + off, len, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaEventRecord(ev[2 * i], s_in) != cudaSuccess || cudaStreamWaitEvent(st, ev[2 * i], 0) != cudaSuccess) {
+      rc = FAVOR_ERR_CUDA;
+      break;
+    }
+    rc = dtype_code == 1
+             ? favor_attention(q8, k8, v8, dom, o8, b1 - b0, H, L, d, M, feature_kind, causal, stream)
+             : favor_attention_f32(reinterpret_cast<float*>(q8), reinterpret_cast<float*>(k8),
+                                   reinterpret_cast<float*>(v8), static_cast<float*>(dom),
+                                   reinterpret_cast<float*>(o8), b1 - b0, H, L, d, M, feature_kind, causal, stream);
+    if (rc != FAVOR_OK) break;
+    issued = i + 1;
+    if (cudaEventRecord(ev[2 * i + 1], st) != cudaSuccess || cudaStreamWaitEvent(s_out, ev[2 * i + 1], 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<uint8_t*>(out) + off, o8, len, cudaMemcpyDeviceToHost, s_out) != cudaSuccess)
       rc = FAVOR_ERR_CUDA;
   }
-  if (rc == FAVOR_OK) {
-    rc = dtype_code == 1
-             ? favor_attention(dq, dk, dv, dom, dout, B, H, L, d, M, feature_kind, causal, stream)
-             : favor_attention_f32(static_cast<float*>(dq), static_cast<float*>(dk), static_cast<float*>(dv),
-                                   static_cast<float*>(dom), static_cast<float*>(dout), B, H, L, d, M,
-                                   feature_kind, causal, stream);
+  (void)issued;
+  // `stream` takes over both copy streams' work before the buffers are released on it
+  if (ev_alloc && ev_done) {
+    if (cudaEventRecord(ev_done, s_in) == cudaSuccess) cudaStreamWaitEvent(st, ev_done, 0);
+    if (cudaEventRecord(ev_done, s_out) == cudaSuccess) cudaStreamWaitEvent(st, ev_done, 0);
   }
-  if (rc == FAVOR_OK && cudaMemcpyAsync(out, dout, nx, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    rc = FAVOR_ERR_CUDA;
   for (void* p : {dq, dk, dv, dom, dout})
     if (p) cudaFreeAsync(p, st);
   if (cudaStreamSynchronize(st) != cudaSuccess && rc == FAVOR_OK) rc = FAVOR_ERR_CUDA;
+  for (int e = 0; e < nev; ++e)
+    if (ev[e]) cudaEventDestroy(ev[e]);
   return rc;
 }
 

@@ -56,3 +56,21 @@ def test_host_buffer_entry_matches_device_entry():
     out = torch.empty_like(hq).pin_memory()
     F.favor_attention_host(hq, hk, hv, hom, out, feature_kind=0)
     assert torch.equal(out, dev)
+
+
+@pytest.mark.parametrize("kind,causal", [(0, False), (1, True), (0, True)])
+def test_host_buffer_entry_pipelines_batch_slices(kind, causal):
+    # B = 6 runs as four batch slices (1, 2, 1, 2 entries) whose copies overlap the compute: each
+    # slice must equal the device entry run on that slice alone
+    import torch
+    import linear_kernelized_attention_b200 as F
+    c = Case(6, 2, 300, 64, 128, seed=12)
+    q, k, v, om = c.device()
+    hq, hk, hv, hom = (t.pin_memory() for t in c.t)
+    out = torch.full_like(hq, float("nan")).pin_memory()
+    F.favor_attention_host(hq, hk, hv, hom, out, feature_kind=kind, causal=causal)
+    for b0, b1 in [(0, 1), (1, 3), (3, 4), (4, 6)]:
+        want = F.favor_attention(q[b0:b1].contiguous(), k[b0:b1].contiguous(), v[b0:b1].contiguous(), om,
+                                 feature_kind=kind, causal=causal).cpu()
+        assert torch.equal(out[b0:b1], want), (b0, b1)
+    assert F.favor_sync_status() == 0
