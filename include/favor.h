@@ -179,7 +179,9 @@ int favor_philox4x64(uint64_t key, uint64_t first_counter, uint64_t n_blocks, ui
  * makes the copies asynchronous). Allocates device buffers from the pool on `stream`, copies
  * in, runs favor_attention (dtype_code 1 = bf16) or favor_attention_f32 (dtype_code 0 =
  * float), copies out and frees. The batch is cut into up to four slices of whole batch entries
- * (slice i = entries [B i / S, B (i+1) / S)): slice i's copies in run on a library-owned
+ * (slice i = entries [B i / S, B (i+1) / S); one slice when an entry's H L d elements are not a
+ * multiple of 16 bytes, since every device entry needs 16-byte aligned pointers): slice i's
+ * copies in run on a library-owned
  * stream, its forward pass on `stream` and its copy out on a second library stream, so one
  * slice's compute and copy out overlap the next slice's copies in; each slice's result equals
  * the device entry run on that slice alone. It synchronises `stream` before returning, so

@@ -818,7 +818,8 @@ int favor_attention_host(const void* q, const void* k, const void* v, const void
   const size_t nx = (size_t)B * per_b, nom = (size_t)H * M * d * es;
   // Batch slices: slice i's copy in, its forward pass and its copy out run on three streams, so
   // one slice's compute and copy out overlap the next slice's copy in.
-  const int S = std::min(B, kHostSlices);
+  // (slices start at whole batch entries; they need the 16-byte alignment every entry point checks)
+  const int S = per_b % 16 == 0 ? std::min(B, kHostSlices) : 1;
   void *dq = nullptr, *dk = nullptr, *dv = nullptr, *dom = nullptr, *dout = nullptr;
   cudaEvent_t ev[2 * kHostSlices + 2] = {};
   const int nev = 2 * S + 2;

@@ -74,3 +74,17 @@ def test_host_buffer_entry_pipelines_batch_slices(kind, causal):
                                  feature_kind=kind, causal=causal).cpu()
         assert torch.equal(out[b0:b1], want), (b0, b1)
     assert F.favor_sync_status() == 0
+
+
+def test_host_buffer_entry_unaligned_batch_entries_run_as_one_slice():
+    # H = 1, L = 50, d = 33 in fp32: a batch entry is 6600 bytes, not a multiple of 16, so the
+    # entry keeps the whole batch in one slice (every device entry needs 16-byte aligned pointers)
+    import torch
+    import linear_kernelized_attention_b200 as F
+    c = Case(3, 1, 50, 33, 40, dtype="f32", seed=13)
+    q, k, v, om = c.device()
+    want = F.favor_attention_f32(q, k, v, om, feature_kind=0).cpu()
+    hq, hk, hv, hom = (t.pin_memory() for t in c.t)
+    out = torch.empty_like(hq).pin_memory()
+    F.favor_attention_host(hq, hk, hv, hom, out, feature_kind=0)
+    assert torch.equal(out, want)
