@@ -277,7 +277,7 @@ int launch_split_t(const SplitPlan& pl, const void* q, const void* k, const void
   sp.meta = meta;
   auto ks = bs::k_bidir_state<KIND, DP>;
   if (ensure_smem_attr(reinterpret_cast<const void*>(ks), pl.k_smem) != FAVOR_OK) return FAVOR_ERR_CUDA;
-  ks<<<pl.Pk, bs::kThreads, pl.k_smem, st>>>(mk, mv, mom, sp);
+  ks<<<pl.Pk, bs::StateCfg<KIND, DP>::kThreads, pl.k_smem, st>>>(mk, mv, mom, sp);
 
   bs::MergeParams mp{};
   mp.nab = pl.nab;

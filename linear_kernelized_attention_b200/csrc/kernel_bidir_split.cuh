@@ -92,6 +92,8 @@ struct StateCfg {
   static constexpr int R = 128 * NSB;                        // state rows of a pair
   static constexpr int NBUF = (KIND == 0 && DP == 128) ? 3 : 5;  // 64-key U/phi buffers
   static constexpr int NS = DP == 64 ? 4 : 2;                // K/V stages
+  static constexpr int NG = KIND == 0 ? 3 : 2;               // feature groups of four warps (trig: SFU-heavy)
+  static constexpr int kThreads = 256 + 128 * NG;             // warps 0-7, then the feature groups
   static constexpr int kStageB = (2 * NCB + 1) * kBoxB;      // V boxes | column box | K boxes
   static constexpr int kOmB = NCB * kBoxB;                   // one Omega block
   static constexpr int kUcol = (NSB * NV + 31) / 32 * 32;    // TMEM column of the U ring
@@ -126,11 +128,11 @@ struct alignas(16) StateMisc {
 static_assert(sizeof(StateMisc) <= 1024, "misc block");
 
 template <int KIND, int DP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(StateCfg<KIND, DP>::kThreads, 1)
     k_bidir_state(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const __grid_constant__ CUtensorMap tm_om, const StateParams p) {
   using C = StateCfg<KIND, DP>;
-  constexpr int NCB = C::NCB, NV = C::NV, NSB = C::NSB, R = C::R, NBUF = C::NBUF, NS = C::NS;
+  constexpr int NCB = C::NCB, NV = C::NV, NSB = C::NSB, R = C::R, NBUF = C::NBUF, NS = C::NS, NG = C::NG;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -181,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   {  // column boxes: zero, with the normaliser column (element 0 of each row) 1.0 for ReLU
     for (int s = 0; s < NS; ++s) {
       uint4* col = reinterpret_cast<uint4*>(gb + (s_stage - base) + s * C::kStageB + NCB * kBoxB);
-      for (int i = tid; i < kBoxB / 16; i += kThreads) col[i] = make_uint4(0u, 0u, 0u, 0u);
+      for (int i = tid; i < kBoxB / 16; i += C::kThreads) col[i] = make_uint4(0u, 0u, 0u, 0u);
     }
     __syncthreads();
     if (KIND == 1 && tid < kTile)
@@ -420,9 +422,55 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nitems = 2 * n;
     bool ok = true;
     RunWalker w(tt0, n, nt);
-    for (int it = g; ok && it < nitems; it += 2) {
+    // Groups 0 and 1 flush share 0 and share 1 of every pair of the run, in pair order: a pair
+    // when the group first reaches an item past it, the last pair after the loop. (Waiting on
+    // s_done for every pair in order keeps each wait within one phase of the barrier.)
+    int flushed = 0;
+    auto flush = [&](int pk) -> bool {
+      const long long pr = p0 + pk;
+      if (!mbar_wait(bar(ms->s_done), pk & 1, abort_flag)) return false;
+      tc_fence_after();
+      float* dst = p.part + slot_of(pr) * (long long)(DP + 1) * R;
+      float mx = 0.f;
+      // trig: group g writes state block g (rows g*128 ..); ReLU: group g writes value
+      // columns [g*DP/2, (g+1)*DP/2) and group 1 the normaliser column
+      const int row = (KIND == 0 ? g * 128 : 0) + q * 32 + lane;
+      const uint32_t sa = tmem + la + (KIND == 0 ? g * NV : 0);
+      const int c_lo = KIND == 0 ? 0 : g * (DP / 2), c_hi = KIND == 0 ? DP : (g + 1) * (DP / 2);
+#pragma unroll 1
+      for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(sa + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float x = __uint_as_float(v[e]);
+          dst[(long long)(c0 + e) * R + row] = x;
+          mx = fmaxf(mx, fabsf(x));
+        }
+      }
+      if (KIND == 0 || g == 1) {
+        uint32_t zc;
+        tmem_ld1(sa + DP, zc);
+        tmem_wait_ld();
+        const float x = __uint_as_float(zc);
+        dst[(long long)DP * R + row] = x;
+        mx = fmaxf(mx, fabsf(x));
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (lane == 0) ms->redmax[pk & 1][g * 4 + q] = mx;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(ms->s_free));
+      return true;
+    };
+    for (int it = g; ok && it < nitems; it += NG) {
       const int t = it >> 1, hf = it & 1, s = t % NS, b = it % NBUF;
       w.advance_to(t);
+      if (g < 2)
+        while (ok && flushed < w.k) ok = flush(flushed++);
+      if (!ok) break;
       if (!(ok = mbar_wait(bar(ms->u_full[b]), (it / NBUF) & 1, abort_flag))) break;
       if (KIND == 0 && hf == 0 && !w.first()) {
         // the tile raised the reference: rescale S once every earlier state MMA has completed
@@ -478,46 +526,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(ms->p_full[b]));
-      if (w.last()) {
-        // flush: this group's share of the state to the pair's workspace slot
-        const int pk = w.k;
-        const long long pr = p0 + pk;
-        if (!(ok = mbar_wait(bar(ms->s_done), pk & 1, abort_flag))) break;
-        tc_fence_after();
-        float* dst = p.part + slot_of(pr) * (long long)(DP + 1) * R;
-        float mx = 0.f;
-        // trig: group g writes state block g (rows g*128 ..); ReLU: group g writes value
-        // columns [g*DP/2, (g+1)*DP/2) and group 1 the normaliser column
-        const int row = (KIND == 0 ? g * 128 : 0) + q * 32 + lane;
-        const uint32_t sa = tmem + la + (KIND == 0 ? g * NV : 0);
-        const int c_lo = KIND == 0 ? 0 : g * (DP / 2), c_hi = KIND == 0 ? DP : (g + 1) * (DP / 2);
-#pragma unroll 1
-        for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld32(sa + c0, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float x = __uint_as_float(v[e]);
-            dst[(long long)(c0 + e) * R + row] = x;
-            mx = fmaxf(mx, fabsf(x));
-          }
-        }
-        if (KIND == 0 || g == 1) {
-          uint32_t zc;
-          tmem_ld1(sa + DP, zc);
-          tmem_wait_ld();
-          const float x = __uint_as_float(zc);
-          dst[(long long)DP * R + row] = x;
-          mx = fmaxf(mx, fabsf(x));
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) ms->redmax[pk & 1][warp - 8] = mx;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(ms->s_free));
-      }
+    }
+    if (g < 2 && ok && n > 0) {
+      w.advance_to(n - 1);
+      while (ok && flushed <= w.k) ok = flush(flushed++);
     }
   }
 
