@@ -506,8 +506,9 @@ int launch_bf16_cuda_cores(const void* q, const void* k, const void* v, const vo
   float* vf = reinterpret_cast<float*>(w8 + 2 * nb);
   float* of = reinterpret_cast<float*>(w8 + 3 * nb);
   float* omf = reinterpret_cast<float*>(w8 + 4 * nb);
-  auto grid = [](long long m) {
-    return (unsigned)std::max<long long>(1, std::min<long long>((m / 8 + 255) / 256, 148ll * 16));
+  const long long max_blocks = 16ll * sm_count();  // grid-stride loops: up to 16 blocks per SM
+  auto grid = [max_blocks](long long m) {
+    return (unsigned)std::max<long long>(1, std::min<long long>((m / 8 + 255) / 256, max_blocks));
   };
   cvt::k_widen<<<grid(n), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), qf, n);
   cvt::k_widen<<<grid(n), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(k), kf, n);
