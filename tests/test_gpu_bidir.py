@@ -48,6 +48,18 @@ def test_bidir_many_heads_single_cta_per_head(kind):
     check_rows(sel, ref, cond, TOL_BF16, U_BIDIR16, f"many heads kind={kind}", trig=kind == 0)
 
 
+@pytest.mark.parametrize("kind", [0, 1])
+@pytest.mark.parametrize("B,H,L", [(4, 64, 128), (2, 128, 256), (1, 30, 384)])
+def test_bidir_runs_crossing_many_short_pairs(kind, B, H, L):
+    # one to three tiles per (head, angle block) pair and up to seven tiles per CTA run, so runs
+    # cross several pair boundaries and a feature group can hold no item of a pair; every row of
+    # every head is checked
+    c = Case(B, H, L, 64, 256, seed=B * 7 + H + L)
+    g = _run(c, kind).reshape(B * H, L, 64)
+    ref, cond, _ = c.oracle(kind, False)
+    check_rows(g, ref, cond, TOL_BF16, U_BIDIR16, f"short pairs kind={kind} {B}x{H}x{L}", trig=kind == 0)
+
+
 def test_bidir_protein_mlm_shape_trig():
     # B=8, H=8, L=1024, d=64, M=256 trig: every row of every head
     c = Case(8, 8, 1024, 64, 256, seed=0)
